@@ -1,0 +1,404 @@
+#!/usr/bin/env python
+"""Benchmark of the rolling-window chunk attention path on B200.
+
+One step = one chunk of one layer, the whole hot path: four denoise reads
+(chunk attention over sinks + window + chunk, with the flow x0 / renoise
+epilogue fused into the output store, sigma = 1.0, 0.75, 0.5, 0.25) and the
+clean t=0 commit (chunk attention plus the K/V write-back into the ring).
+RoPE (relative or absolute) runs on the way in. Inputs are synthetic (seeded
+counter-based generator), resident in HBM before timing; the cache is rolled
+to steady state (full window, evictions firing) before warm-up.
+
+Metric: query tokens / s per layer (5 * Lq per step), whole job over all ranks.
+Multi-GPU: independent replicas (one layer each), no data-path collective.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config abot|480p|720p] [--impl rkv|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "query tokens/s per layer; attn TFLOP/s as % of B200 dense BF16 peak"
+UNIT = "query tokens/s"
+
+CONFIGS = {
+    "abot": dict(workload="ABot-style relative RoPE: 1 layer, H=24, d=128, 880 tokens/frame (22x40 grid), "
+                          "chunk 3 frames (2640 queries), window 21 frames (18480 keys), 5 sink reference frames, "
+                          "4 denoise reads (fused x0/renoise) + 1 commit per chunk",
+                 H=24, gh=22, gw=40, C=3, W=21, S=5, refs=5, mode=1),
+    "480p": dict(workload="LingBot-style 480P: 1 layer, H=40, d=128, 1560 tokens/frame (30x52 grid), chunk 4 frames "
+                          "(6240 queries), window 18 frames (28080 keys), sink 6, absolute RoPE, "
+                          "4 denoise reads (fused x0/renoise) + 1 commit per chunk",
+                 H=40, gh=30, gw=52, C=4, W=18, S=6, refs=0, mode=0),
+    "720p": dict(workload="720p: 1 layer, H=40, d=128, 3600 tokens/frame (45x80 grid), chunk 4 frames (14400 queries), "
+                          "window 18 frames (64800 keys), sink 6, absolute RoPE, fused x0/renoise on the "
+                          "[14400 x 5120] latent, 4 denoise reads + 1 commit per chunk",
+                 H=40, gh=45, gw=80, C=4, W=18, S=6, refs=0, mode=0),
+}
+SIGMAS = [1.0, 0.75, 0.5, 0.25]
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            p = json.load(fh)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str | None):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+        if gpu_id is None:
+            return
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", gpu_id, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as fh:
+            for line in fh:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 8:
+                    continue
+                try:
+                    sm.append(float(parts[0]))
+                    mx = float(parts[1])
+                except ValueError:
+                    continue
+                for n, val in zip(names, parts[4:8]):
+                    if val.lower() == "active":
+                        reasons.add(n)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------- CUDA arm
+def visible_keys(cfg, committed, f0):
+    import rolling_kv_chunked_b200 as rkv
+    T = cfg["gh"] * cfg["gw"]
+    return sum(n for _, _, n, _ in rkv.plan_window(cfg["W"], cfg["S"], committed, cfg["C"], f0)) * T
+
+
+def run_rkv(args):
+    import torch
+    import torch.distributed as dist
+
+    import rolling_kv_chunked_b200 as rkv
+    import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
+
+    cfg = CONFIGS[args.config]
+    H, C, W, S = cfg["H"], cfg["C"], cfg["W"], cfg["S"]
+    T = cfg["gh"] * cfg["gw"]
+    Lq = C * T
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+    h = rkv.RollingKV(1, H, 128, T, W, S, cfg["mode"])
+    h.set_rope_grid(cfg["gh"], cfg["gw"])
+
+    def fill(t, *fields):
+        synth.fill_normal_bf16_cuda(t.data_ptr(), t.numel(), synth.stream_key(rank, 77, *fields), 0, sp)
+        return t
+
+    bf = dict(dtype=torch.bfloat16, device="cuda")
+    # a pool of step input sets (inputs of one step are ~300 MB, larger than L2)
+    pool_n = 2
+    pool = []
+    for i in range(pool_n):
+        pool.append(dict(
+            q=[fill(torch.empty((Lq, H, 128), **bf), i, c, 1) for c in range(5)],
+            k=[fill(torch.empty((Lq, H, 128), **bf), i, c, 2) for c in range(5)],
+            v=[fill(torch.empty((Lq, H, 128), **bf), i, c, 3) for c in range(5)],
+            xt=fill(torch.empty((Lq, H * 128), **bf), i, 9, 4),
+            eps=[fill(torch.empty((Lq, H * 128), **bf), i, c, 5) for c in range(3)],
+        ))
+    outs = [torch.empty((Lq, H, 128), **bf) for _ in range(5)]
+    x0 = torch.empty((Lq, H * 128), **bf)
+    xn = [torch.empty((Lq, H * 128), **bf) for _ in range(2)]
+    state = {"f0": 0}
+
+    def step(inp):
+        f0 = state["f0"]
+        xt = inp["xt"]
+        for s in range(4):
+            sn = SIGMAS[s + 1] if s < 3 else -1.0
+            nxt = xn[s % 2] if sn >= 0 else None
+            h.chunk_attention(0, inp["q"][s], inp["k"][s], inp["v"][s], outs[s], C, f0, False, stream=sp,
+                              flow=dict(xt=xt, eps=inp["eps"][s] if sn >= 0 else None, sigma=SIGMAS[s],
+                                        sigma_next=sn, x0_out=x0, xt_next_out=nxt))
+            if nxt is not None:
+                xt = nxt
+        h.chunk_attention(0, inp["q"][4], inp["k"][4], inp["v"][4], outs[4], C, f0, True, stream=sp)
+        state["f0"] = f0 + C
+
+    # reference frames (sinks) and roll the window to steady state
+    if cfg["refs"]:
+        kr = fill(torch.empty((cfg["refs"] * T, H, 128), **bf), 99, 0, 2)
+        vr = fill(torch.empty((cfg["refs"] * T, H, 128), **bf), 99, 0, 3)
+        h.write_chunk(0, kr, vr, cfg["refs"], 0, stream=sp)
+        state["f0"] = cfg["refs"]
+    prefill = math.ceil((W - S) / C) + 1
+    for i in range(prefill):
+        inp = pool[i % pool_n]
+        h.chunk_attention(0, inp["q"][4], inp["k"][4], inp["v"][4], outs[4], C, state["f0"], True, stream=sp)
+        state["f0"] += C
+    for i in range(args.warmup):
+        step(pool[i % pool_n])
+    torch.cuda.synchronize()
+    if h.poll_device_status(sp) != rkv.OK:
+        raise RuntimeError("device wait expired during warm-up")
+
+    # FLOPs of the attention launches in the timed region (unmasked visible keys)
+    flops = 0.0
+    f = state["f0"]
+    for _ in range(args.steps):
+        flops += 5 * 4.0 * H * 128 * Lq * visible_keys(cfg, f, f)
+        f += C
+
+    gpu_id = None
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
+    except Exception:
+        gpu_id = None
+    clocks = ClockSampler(gpu_id)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    h.timing_begin(5 * args.steps)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for i in range(args.steps):
+        step(pool[i % pool_n])
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    kernel_ms = h.timing_end(5 * args.steps)
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = ev0.elapsed_time(ev1)
+    status = h.poll_device_status(sp)
+    if status != rkv.OK:
+        raise RuntimeError("device wait expired in the timed region")
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    tokens = 5 * Lq * args.steps * world
+    value = tokens / (ms / 1e3)
+
+    # ---- end to end through the C ABI with host buffers (copies inside the timed region)
+    hostset = []
+    for i in range(2):
+        src = pool[i]
+        hostset.append({k: ([t.cpu().pin_memory() for t in v] if isinstance(v, list) else v.cpu().pin_memory())
+                        for k, v in src.items()})
+    dev = pool[0]
+    host_out = [torch.empty((Lq, H, 128), dtype=torch.bfloat16).pin_memory() for _ in range(5)]
+    host_x0 = torch.empty((Lq, H * 128), dtype=torch.bfloat16).pin_memory()
+    h2d = sum(t.numel() * 2 for k, v in hostset[0].items() for t in (v if isinstance(v, list) else [v]))
+    d2h = sum(t.numel() * 2 for t in host_out) + host_x0.numel() * 2
+
+    def e2e_step(i):
+        hs = hostset[i % 2]
+        for key_, val in hs.items():
+            if isinstance(val, list):
+                for d_, s_ in zip(dev[key_], val):
+                    d_.copy_(s_, non_blocking=True)
+            else:
+                dev[key_].copy_(val, non_blocking=True)
+        step(dev)
+        for d_, s_ in zip(host_out, outs):
+            d_.copy_(s_, non_blocking=True)
+        host_x0.copy_(x0, non_blocking=True)
+
+    e2e_step(0)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        e2e_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = tokens / (e2e_ms / 1e3)
+
+    pk, pk_kind = peaks()
+    mean_kernel_ms = sum(kernel_ms) / max(1, len(kernel_ms))
+    achieved = flops / (sum(kernel_ms) / 1e3) / 1e12 if kernel_ms else None
+    peak = pk["bf16_tflops_sustained"]
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": cfg["workload"], "queries_per_call": Lq, "keys_per_call": W * T,
+                   "calls_per_step": 5, "parallelism": f"replicas x{world} (no data-path collective)",
+                   "l2": f"inputs larger than L2 ({(15 * Lq * H * 128 + 4 * Lq * H * 128) * 2 / 1e6:.0f} MB per step)"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": (achieved / peak) if achieved else None, "traffic": None,
+                     "kernel": "chunk_attention_kernel", "peak_source": f"{pk_kind} bf16_tflops_sustained",
+                     "frac_of_burst": (achieved / pk["bf16_tflops"]) if achieved else None,
+                     "mean_kernel_ms": mean_kernel_ms, "launches_timed": len(kernel_ms),
+                     "flops_per_launch": flops / max(1, 5 * args.steps)},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 11 * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(cfg, budget_s=args.cpu_seconds)
+    h.close()
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+# ---------------------------------------------------------------------- oracle arm
+def _oracle_steady_layer(cfg):
+    """An oracle layer holding a full steady-state window (one synthetic frame reused)."""
+    import synth
+    from oracle.layer import OracleLayer
+    H, C, W, S = cfg["H"], cfg["C"], cfg["W"], cfg["S"]
+    T = cfg["gh"] * cfg["gw"]
+    orc = OracleLayer(H, 128, T, cfg["gh"], cfg["gw"], W, S, cfg["mode"])
+    frame = synth.normal_bf16_bits(synth.stream_key(0, 78), 0, T * H * 128).reshape(T, H, 128)
+    f = 0
+    while f < W + C:
+        orc.write_chunk(frame, frame, 1, f)
+        f += 1
+    q = synth.normal_bf16_bits(synth.stream_key(0, 79), 0, C * T * H * 128).reshape(C * T, H, 128)
+    return orc, q, f
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max(i.get("num_threads", 1) for i in threadpool_info()) or os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(cfg, budget_s=10.0, heads=2):
+    """The oracle as it stands, on a bounded sample: `heads` of H heads of steady-state
+    denoise reads (all queries, full window), repeated for ~budget_s, scaled by H / heads."""
+    orc, q, f0 = _oracle_steady_layer(cfg)
+    C, H = cfg["C"], cfg["H"]
+    T = cfg["gh"] * cfg["gw"]
+    n, t0 = 0, time.perf_counter()
+    while True:
+        orc.chunk_attention(q, q, q, C, f0, False, heads=list(range(heads)))
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    per_call_s = el / n * (H / heads)
+    return {"value": C * T / per_call_s, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"{n} steady-state reads x {heads} of {H} heads (all {C * T} queries vs {cfg['W'] * T} keys), "
+                      f"numpy fp64, scaled by {H}/{heads}"}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    cfg = CONFIGS[args.config]
+    orc, q, f0 = _oracle_steady_layer(cfg)
+    C, H = cfg["C"], cfg["H"]
+    T = cfg["gh"] * cfg["gw"]
+    Lq = C * T
+    heads = [0]
+    for _ in range(args.warmup):
+        orc.chunk_attention(q, q, q, C, f0, False, heads=heads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        orc.chunk_attention(q, q, q, C, f0, False, heads=heads)
+    el = time.perf_counter() - t0
+    per_call_s = el / args.steps * H
+    value = Lq / per_call_s
+    sample = (f"each step: one steady-state read, 1 of {H} heads (all {Lq} queries vs {cfg['W'] * T} keys), "
+              f"scaled by {H}")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": cfg["workload"]},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="abot", choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="rkv", choices=["rkv", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_rkv(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,209 @@
+/*
+ * rkv.h - C ABI of librkv.so: block-causal chunk attention over a fixed-size
+ * rolling KV cache with never-evicted sink frames, 3D RoPE (absolute or
+ * relative), the clean t=0 K/V write-back, and the flow-matching x0/renoise
+ * epilogue, as hand-written sm_100a (B200) CUDA kernels.
+ *
+ * Pages cited by title and section:
+ *  [P1] "LingBot-World 2.0因果预训练范式深度剖析：为什么它能持续生成视频而不“掉画质”"
+ *       (sheratonhq.com/news/156439)
+ *  [P2] "从40步到4步：LingBot-World 2.0实时推理蒸馏（causal_fast）原理与关键代码解读"
+ *       (hmyw.cn/news/135683)
+ *  [P3] LingBot-World 2.0 wan/ source-map article (kwkr.cn/news/564388)
+ *  [P4] "ABot-World流式因果推理深度解析：KV缓存与块级注意力如何让24小时连续生成不漂移"
+ *       (lpnh.cn/news/2488095)
+ *
+ * Conventions for every call:
+ *  - Tensors are bf16, contiguous, token-major: [tokens, H, d] with tokens
+ *    ordered frame, then latent grid row, then grid column. d must be 128.
+ *  - Pointers named q/k/v/out/x/xt/eps/x0_out/xt_next_out are DEVICE
+ *    pointers owned by the caller; they must be 16-byte aligned. The library
+ *    never frees them and keeps no reference after the call returns.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream). Every device launch is asynchronous on that stream; host state
+ *    (frames committed, slot map) advances when the call is enqueued.
+ *  - Calls on one handle must be issued from one host thread and, for a given
+ *    layer, be ordered on one stream (the per-layer scratch is reused).
+ *  - Return value: RKV_OK or one of the RKV_ERR_* codes below. Argument,
+ *    order and capacity errors are detected on the host before anything is
+ *    launched; then no state changes.
+ */
+#ifndef RKV_H_
+#define RKV_H_
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define RKV_OK 0
+#define RKV_ERR_ARG 1         /* bad pointer, size, layer index or alignment            */
+#define RKV_ERR_ORDER 2       /* start_frame != frames committed so far for that layer  */
+#define RKV_ERR_CAPACITY 3    /* n_frames > window_frames - sink_frames                 */
+#define RKV_ERR_UNSUPPORTED 4 /* d != 128, window > 256 frames, time id beyond table    */
+#define RKV_ERR_CUDA 5        /* a CUDA runtime / driver call failed                    */
+#define RKV_ERR_TIMEOUT 6     /* a bounded device wait expired (read via poll)          */
+#define RKV_ERR_STATE 7       /* call needs rkv_set_rope_grid first                     */
+
+#define RKV_ROPE_ABSOLUTE 0   /* time id = absolute frame index                         */
+#define RKV_ROPE_RELATIVE 1   /* time id re-based to the window and clamped to [0, W-1] */
+
+typedef struct rkv_ctx* rkv_handle;
+
+/*
+ * rkv_create - allocate the per-layer rolling caches.
+ *  Window of `window_frames` frames ([P1] §滑动窗口 KV 缓存 local_attn_size; [P4] §机制一
+ *  cache size local_attn_size x tokens per frame), of which the first
+ *  `sink_frames` frames ever written are never evicted ([P1] §Attention Sink sink_size;
+ *  [P4] §机制一 reference-view sinks). `tokens_per_frame` = T; `rope_mode` is
+ *  RKV_ROPE_ABSOLUTE or RKV_ROPE_RELATIVE ([P3] §改造③ start_frame; [P4] §机制三).
+ *  Device memory per layer (library-owned, freed by rkv_destroy, zero-filled):
+ *  raw K and V rings [H][window*T][d], a rotated-K ring plus chunk area
+ *  [H][(2*window - sink)*T][d] and a rotated-Q staging area [H][(window-sink)*T][d].
+ *  Errors: RKV_ERR_ARG (non-positive sizes, sink >= window, null out),
+ *  RKV_ERR_UNSUPPORTED (d != 128, window_frames > 256), RKV_ERR_CUDA (allocation).
+ */
+int rkv_create(int layers, int H, int d, int tokens_per_frame, int window_frames,
+               int sink_frames, int rope_mode, rkv_handle* out);
+
+/*
+ * rkv_set_rope_grid - the latent grid and rotary layout (required before any
+ *  call that rotates). grid_h * grid_w must equal tokens_per_frame; token i of
+ *  a frame sits at row i / grid_w, column i % grid_w. The d/2 adjacent pairs
+ *  (x[2p], x[2p+1]) are split pairs_t (time), pairs_h (row), pairs_w (column),
+ *  in that order; pair j of an axis with n pairs turns by pos * theta^(-j/n).
+ *  cos/sin tables are built on the host in double and stored as fp32.
+ *  Errors: RKV_ERR_ARG (grid mismatch, pairs_t+pairs_h+pairs_w != d/2, theta <= 0).
+ */
+int rkv_set_rope_grid(rkv_handle h, int grid_h, int grid_w, double theta,
+                      int pairs_t, int pairs_h, int pairs_w);
+
+/*
+ * rkv_write_chunk - commit `n_frames` frames of raw K/V ([n_frames*T, H, d]) to
+ *  `layer` without attending (e.g. the five reference views that become the
+ *  sinks, [P4] §一次流式生成 / §机制一). start_frame must equal the frames
+ *  committed so far. Eviction follows [P2] §3: frames after the sinks are
+ *  dropped oldest first. Errors: RKV_ERR_ARG, RKV_ERR_ORDER, RKV_ERR_CAPACITY,
+ *  RKV_ERR_STATE (absolute mode needs the grid), RKV_ERR_CUDA.
+ */
+int rkv_write_chunk(rkv_handle h, int layer, const void* k, const void* v,
+                    int n_frames, int start_frame, void* stream);
+
+/*
+ * rkv_chunk_attention - O = softmax(RoPE(Q) RoPE(K)^T / sqrt(d)) V for the
+ *  chunk [start_frame, start_frame + n_frames) of `layer`: the chunk's queries
+ *  see the sinks, the latest committed history that still fits the window, and
+ *  the chunk itself, with no mask inside that set ([P2] §3 window slice then
+ *  attention(roped_query, k_cache, v_cache); [P4] §机制二 block-causal mask).
+ *  q, k, v, out: [n_frames*T, H, d]. commit = 0: a denoise read, the cache is
+ *  unchanged. commit = 1: the clean t=0 pass ([P2] §3; [P4] §机制二 干净上下文回写):
+ *  same attention, then k/v are written into the ring (raw K in both modes).
+ *  Errors: RKV_ERR_ARG, RKV_ERR_ORDER, RKV_ERR_CAPACITY, RKV_ERR_STATE,
+ *  RKV_ERR_UNSUPPORTED (absolute time id >= 65536), RKV_ERR_CUDA.
+ */
+int rkv_chunk_attention(rkv_handle h, int layer, const void* q, const void* k, const void* v,
+                        void* out, int n_frames, int start_frame, int commit, void* stream);
+
+/*
+ * Flow-matching epilogue fused into the attention output store: the attention
+ *  output (rounded to bf16, exactly the value written to `out`) is taken as the
+ *  flow prediction v of the latent [n_frames*T, H*d] and the epilogue of
+ *  rkv_flow_x0_renoise is applied to it in the same kernel. Fields as there.
+ */
+typedef struct {
+  const void* xt;        /* [n_frames*T, H*d] bf16, current noisy latent        */
+  const void* eps;       /* [n_frames*T, H*d] bf16, noise for the renoise step  */
+  double sigma;          /* sigma of this step                                  */
+  double sigma_next;     /* next sigma; < 0 marks the last step (no renoise)    */
+  void* x0_out;          /* [n_frames*T, H*d] bf16 out                          */
+  void* xt_next_out;     /* [n_frames*T, H*d] bf16 out; may be NULL on last step */
+} rkv_flow_epilogue;
+
+/* rkv_chunk_attention_flow - rkv_chunk_attention plus the fused epilogue
+ *  (`epi` NULL = no epilogue). Errors as rkv_chunk_attention. */
+int rkv_chunk_attention_flow(rkv_handle h, int layer, const void* q, const void* k,
+                             const void* v, void* out, int n_frames, int start_frame,
+                             int commit, const rkv_flow_epilogue* epi, void* stream);
+
+/*
+ * rkv_rope_apply - rotate x [n_frames*T, H, d] in place with the handle's 3D
+ *  RoPE. Absolute mode: t = frame index ([P3] §改造③ rope_apply(..., start_frame)).
+ *  Relative mode: t = clamp(f - (window_end_frame - window_frames), 0, W-1),
+ *  window_end_frame = one past the last frame of the window ([P4] §机制三);
+ *  ignored in absolute mode. fp32 arithmetic, bf16 round-to-nearest-even out.
+ *  Errors: RKV_ERR_ARG, RKV_ERR_STATE, RKV_ERR_UNSUPPORTED, RKV_ERR_CUDA.
+ */
+int rkv_rope_apply(rkv_handle h, void* x, int n_frames, int start_frame,
+                   int window_end_frame, void* stream);
+
+/*
+ * rkv_flow_x0_renoise - x0 = xt - sigma * v; if sigma_next >= 0 also
+ *  xt_next = (1 - sigma_next) * x0 + sigma_next * eps ([P2] §2 _convert_flow_pred_to_x0
+ *  and re-noise to the next timestep; §精度 flow->x0 in double). n elements,
+ *  bf16 in/out, fp64 arithmetic without fused multiply-add, round-to-nearest-even
+ *  on output; renoise uses the unrounded fp64 x0. eps / xt_next_out may be NULL
+ *  when sigma_next < 0. Errors: RKV_ERR_ARG, RKV_ERR_CUDA.
+ */
+int rkv_flow_x0_renoise(const void* xt, const void* v, const void* eps, double sigma,
+                        double sigma_next, void* x0_out, void* xt_next_out, long long n,
+                        void* stream);
+
+/* rkv_slot_frames - host copy of the slot -> frame map of `layer`: frames_out[W],
+ *  -1 = empty. Slots [0, S) hold the sinks; frame f >= S lives in slot
+ *  S + (f - S) mod (W - S). Errors: RKV_ERR_ARG. */
+int rkv_slot_frames(rkv_handle h, int layer, int* frames_out);
+
+/* rkv_frames_committed - frames committed so far to `layer`. Errors: RKV_ERR_ARG. */
+int rkv_frames_committed(rkv_handle h, int layer, int* out);
+
+/* rkv_cache_ptrs - device pointers of the raw K and V rings of `layer`, each
+ *  [H][W*T][d] bf16 with slot s at rows [s*T, (s+1)*T). Library-owned, valid
+ *  until rkv_destroy; for read-back only. Errors: RKV_ERR_ARG. */
+int rkv_cache_ptrs(rkv_handle h, int layer, void** k, void** v);
+
+/* rkv_reset - forget all frames of every layer and zero the caches (synchronous).
+ *  Errors: RKV_ERR_ARG, RKV_ERR_CUDA. */
+int rkv_reset(rkv_handle h);
+
+/* rkv_destroy - free everything the handle owns (synchronises the device). */
+int rkv_destroy(rkv_handle h);
+
+/* rkv_status_string - static text for a status code. */
+const char* rkv_status_string(int status);
+
+/* rkv_poll_device_status - synchronise `stream`, read and clear the handle's
+ *  device status word. RKV_ERR_TIMEOUT if a kernel's bounded wait expired since
+ *  the last poll (that kernel stopped early and its output is invalid). */
+int rkv_poll_device_status(rkv_handle h, void* stream);
+
+/* rkv_set_wait_limit - cap, in nanoseconds, on each bounded device wait of the
+ *  attention kernel's main loop (default 2e9). Diagnostic: a tiny cap makes the
+ *  wait expire so the timeout path can be tested. Errors: RKV_ERR_ARG. */
+int rkv_set_wait_limit(rkv_handle h, long long nanoseconds);
+
+/* rkv_timing_begin - start recording a CUDA event pair around each attention
+ *  kernel launch (on the caller's stream), for at most max_launches launches.
+ *  Instrumentation only: nothing is skipped. Errors: RKV_ERR_ARG, RKV_ERR_CUDA. */
+int rkv_timing_begin(rkv_handle h, int max_launches);
+
+/* rkv_timing_end - synchronise the recorded events, write the duration (ms) of
+ *  each recorded attention launch to ms_out[0 .. *n_out) (at most max) and stop
+ *  recording. Errors: RKV_ERR_ARG, RKV_ERR_CUDA. */
+int rkv_timing_end(rkv_handle h, float* ms_out, int max, int* n_out);
+
+/*
+ * rkv_plan_window - host-only planner (no GPU needed): the key segments that
+ *  chunk [start_frame, start_frame + n_frames) attends to, in logical order,
+ *  given `frames_committed` frames already in a window of W frames with S sinks.
+ *  Writes up to max_segs records of 4 ints to seg_out:
+ *    {source (0 = ring slots, 1 = the call's own chunk), first slot (source 0) or
+ *     first chunk frame (source 1), number of frames, absolute id of the first frame}
+ *  and their count to *n_segs. Errors: RKV_ERR_ARG, RKV_ERR_ORDER, RKV_ERR_CAPACITY.
+ */
+int rkv_plan_window(int window_frames, int sink_frames, int frames_committed, int n_frames,
+                    int start_frame, int* seg_out, int max_segs, int* n_segs);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RKV_H_ */

@@ -1,0 +1,44 @@
+// bf16 <-> fp32/fp64 helpers shared by the kernels.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+
+namespace rkv {
+
+__device__ __forceinline__ float bf16_to_f32(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
+
+__device__ __forceinline__ uint16_t f32_to_bf16_rne(float x) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+
+// fp64 -> bf16, round to nearest even, without double rounding: first round
+// toward zero to fp32 and set the last fp32 bit when anything was dropped
+// ("round to odd"), then round that fp32 to bf16 to nearest even. Rounding to
+// odd in a format with at least two more bits than the target, followed by
+// round-to-nearest, gives the correctly rounded result (Boldo & Melquiond,
+// "Emulation of FMA and correctly rounded sums: proved algorithms using
+// rounding to odd", IEEE Trans. Computers 57(4), 2008). fp32 keeps 16 more
+// significand bits than bf16, in the normal and the subnormal range alike.
+__device__ __forceinline__ uint16_t f64_to_bf16_rne(double x) {
+  const float f = __double2float_rz(x);
+  uint32_t u = __float_as_uint(f);
+  if (static_cast<double>(f) != x) u |= 1u;
+  u = (u + 0x7FFFu + ((u >> 16) & 1u)) >> 16;
+  return static_cast<uint16_t>(u);
+}
+
+// x0 = xt - sigma * v; xt' = (1 - sigma') * x0 + sigma' * eps, in fp64 with every
+// operation rounded on its own (no fused multiply-add).
+struct FlowStep {
+  double sigma, one_minus_next, sigma_next;
+  bool renoise;
+  __device__ __forceinline__ void apply(double xt, double v, double eps, uint16_t& x0_out,
+                                        uint16_t& xn_out) const {
+    const double x0 = __dsub_rn(xt, __dmul_rn(sigma, v));
+    x0_out = f64_to_bf16_rne(x0);
+    if (renoise) xn_out = f64_to_bf16_rne(__dadd_rn(__dmul_rn(one_minus_next, x0), __dmul_rn(sigma_next, eps)));
+  }
+};
+
+}  // namespace rkv

@@ -1,0 +1,391 @@
+// Chunk attention over the rolling window on sm_100a (K2).
+//
+// O = softmax(Q K^T / sqrt(d)) V for one chunk's queries against the logical key
+// stream "sinks, ring run 1, ring run 2 (wrap), current chunk" (up to four
+// segments). Block-causal at chunk granularity means there is no mask inside
+// that stream ("ABot-World流式因果推理深度解析", §机制二: a new block's queries see
+// their own block plus the history blocks of the window, frames inside a block see
+// each other; "从40步到4步：LingBot-World 2.0实时推理蒸馏（causal_fast）原理与关键代码
+// 解读", §3: window slice then attention(roped_query, k_cache, v_cache)). Keys
+// outside the window are never loaded, so masked tiles are never issued; the
+// only masking is of the ragged last tile of each segment.
+//
+// Queries and keys arrive already rotated (RoPE applied by the frame-run kernel on
+// their way into the head-major staging / rotated-K ring), V raw.
+//
+// Structure of one CTA (one head, 256 query rows = two 128-row tiles Q0, Q1):
+//   warps 0-3  softmax for Q0 (one thread per query row = TMEM lane)
+//   warps 4-7  softmax for Q1
+//   warp 8     TMA producer: Q0/Q1 once, then K and V tiles (128 keys) into a
+//              2-stage ring each
+//   warp 9     TMEM allocator and tcgen05.mma issuer (one thread)
+// TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each; the bf16
+// probabilities P overwrite the first 64 columns of their S tile and feed the PV
+// product straight from TMEM. MMA issue order per key tile j:
+//   S0(j) = Q0 K_j^T, PV1(j-1), S1(j) = Q1 K_j^T, PV0(j)
+// so that while one softmax warpgroup works on its tile the tensor core runs the
+// other tile's products. Online softmax in the log2 domain with a lazy rescale
+// (O is rescaled only when a row maximum grows by more than 2^8).
+//
+// Every mbarrier wait is bounded in wall time; on expiry the kernel records
+// kStatusTimeout in the status word, stops issuing work, waits (bounded) for the
+// copies and MMAs it already issued, frees TMEM and returns.
+#include <cfloat>
+
+#include "numeric.cuh"
+#include "ptx_sm100.cuh"
+#include "rkv_internal.h"
+
+namespace rkv {
+namespace {
+
+constexpr int kBM = 128;                  // query rows per tile (TMEM lanes)
+constexpr int kBN = 128;                  // keys per tile
+constexpr int kSlab = 128 * 64 * 2;       // 128 rows x 64 bf16, one 128-byte swizzle span per row
+constexpr int kTile = 2 * kSlab;          // 128 rows x 128 bf16
+constexpr int kThreads = 320;
+constexpr int kSmemQ = 0;                 // Q0, Q1
+constexpr int kSmemK = 2 * kTile;         // K stage 0, 1
+constexpr int kSmemV = 4 * kTile;         // V stage 0, 1
+constexpr int kSmemBar = 6 * kTile;
+constexpr int kSmemBytes = 6 * kTile + 256 + 1024;  // tiles + barriers + alignment slack
+constexpr unsigned long long kDrainNs = 2000000000ull;
+
+enum : int {
+  kBarQ = 0,
+  kBarKFull = 1,   // +stage
+  kBarKEmpty = 3,  // +stage
+  kBarVFull = 5,   // +stage
+  kBarVEmpty = 7,  // +stage
+  kBarSFull = 9,   // +tile (0, 1)
+  kBarPFull = 11,  // +tile
+  kBarODone = 13,
+  kBarDrain = 14,
+  kNumBars = 15
+};
+
+// TMEM column of the S / P tile and of the O accumulator of query tile t (0 or 1).
+__device__ __forceinline__ constexpr uint32_t col_s(int t) { return static_cast<uint32_t>(t) * 128u; }
+__device__ __forceinline__ constexpr uint32_t col_o(int t) { return 256u + static_cast<uint32_t>(t) * 128u; }
+constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(kBM, kBN, false);        // K-major A and B
+constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(kBM, kHeadDim, true);   // B (V) MN-major
+
+__device__ __forceinline__ void tile_of(const AttnParams& p, int j, int& src, int& krow, int& vrow,
+                                        int& valid) {
+  int t = j;
+#pragma unroll
+  for (int s = 0; s < kMaxSegs; ++s) {
+    if (s < p.n_segs) {
+      const int nt = (p.seg[s].n_rows + kBN - 1) / kBN;
+      if (t < nt) {
+        src = p.seg[s].src;
+        krow = p.seg[s].k_row0 + t * kBN;
+        vrow = p.seg[s].v_row0 + t * kBN;
+        valid = min(kBN, p.seg[s].n_rows - t * kBN);
+        return;
+      }
+      t -= nt;
+    }
+  }
+  src = 0;
+  krow = vrow = 0;
+  valid = 0;
+}
+
+// K-major operand (Q or K tile): k-step kk covers elements [16kk, 16kk+16) of every row.
+__device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile_addr, int kk) {
+  return ptx::smem_desc_sw128(tile_addr + (kk >> 2) * kSlab + (kk & 3) * 32, 16, 1024);
+}
+
+// MN-major operand (V tile as B of O += P V): k-step kk covers keys [16kk, 16kk+16);
+// the two 64-column halves of d are kSlab apart.
+__device__ __forceinline__ uint64_t desc_v(uint32_t tile_addr, int kk) {
+  return ptx::smem_desc_sw128(tile_addr + kk * 2048, kSlab, 1024);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  return static_cast<uint32_t>(f32_to_bf16_rne(lo)) | (static_cast<uint32_t>(f32_to_bf16_rne(hi)) << 16);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    chunk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                           const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_vn,
+                           const __grid_constant__ AttnParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSmemBar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int head = blockIdx.y;
+  const int m0 = blockIdx.x * (2 * kBM);
+  const unsigned long long limit = p.wait_limit_ns;
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&bars[kBarQ], 1);
+    for (int s = 0; s < 2; ++s) {
+      ptx::mbar_init(&bars[kBarKFull + s], 1);
+      ptx::mbar_init(&bars[kBarKEmpty + s], 1);
+      ptx::mbar_init(&bars[kBarVFull + s], 1);
+      ptx::mbar_init(&bars[kBarVEmpty + s], 1);
+      ptx::mbar_init(&bars[kBarSFull + s], 1);
+      ptx::mbar_init(&bars[kBarPFull + s], kBM);
+    }
+    ptx::mbar_init(&bars[kBarODone], 1);
+    ptx::mbar_init(&bars[kBarDrain], 1);
+    ptx::fence_mbar_init();
+  }
+  if (warp == 9) {
+    ptx::tmem_alloc(tmem_slot, 512);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int n_tiles = p.n_tiles;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      ptx::prefetch_tmap(&tm_q);
+      ptx::prefetch_tmap(&tm_k);
+      ptx::prefetch_tmap(&tm_vc);
+      ptx::prefetch_tmap(&tm_vn);
+      ptx::mbar_arrive_expect_tx(&bars[kBarQ], 2 * kTile);
+      for (int t = 0; t < 2; ++t)
+        for (int c = 0; c < 2; ++c)
+          ptx::tma_load_3d(smem + kSmemQ + t * kTile + c * kSlab, &tm_q, &bars[kBarQ], c * 64, m0 + t * kBM, head);
+      bool ok = true;
+      int nk = 0, nv = 0;
+      for (int j = 0; j < n_tiles; ++j) {
+        const int s = j & 1;
+        int src, krow, vrow, valid;
+        tile_of(p, j, src, krow, vrow, valid);
+        if (j >= 2 && !ptx::mbar_wait(&bars[kBarKEmpty + s], ((j - 2) >> 1) & 1, limit)) { ok = false; break; }
+        ptx::mbar_arrive_expect_tx(&bars[kBarKFull + s], kTile);
+        for (int c = 0; c < 2; ++c)
+          ptx::tma_load_3d(smem + kSmemK + s * kTile + c * kSlab, &tm_k, &bars[kBarKFull + s], c * 64, krow, head);
+        nk = j + 1;
+        if (j >= 2 && !ptx::mbar_wait(&bars[kBarVEmpty + s], ((j - 2) >> 1) & 1, limit)) { ok = false; break; }
+        ptx::mbar_arrive_expect_tx(&bars[kBarVFull + s], kTile);
+        for (int c = 0; c < 2; ++c) {
+          if (src == 0)
+            ptx::tma_load_3d(smem + kSmemV + s * kTile + c * kSlab, &tm_vc, &bars[kBarVFull + s], c * 64, vrow, head);
+          else
+            ptx::tma_load_3d(smem + kSmemV + s * kTile + c * kSlab, &tm_vn, &bars[kBarVFull + s], c * 64, head, vrow);
+        }
+        nv = j + 1;
+      }
+      if (!ok) atomicOr(p.status, kStatusTimeout);
+      // every copy issued must land before the CTA may exit
+      ptx::mbar_wait(&bars[kBarQ], 0, kDrainNs);
+      for (int j = (nk > 2 ? nk - 2 : 0); j < nk; ++j) ptx::mbar_wait(&bars[kBarKFull + (j & 1)], (j >> 1) & 1, kDrainNs);
+      for (int j = (nv > 2 ? nv - 2 : 0); j < nv; ++j) ptx::mbar_wait(&bars[kBarVFull + (j & 1)], (j >> 1) & 1, kDrainNs);
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t q_addr[2] = {ptx::smem_u32(smem + kSmemQ), ptx::smem_u32(smem + kSmemQ + kTile)};
+      const uint32_t k_addr = ptx::smem_u32(smem + kSmemK);
+      const uint32_t v_addr = ptx::smem_u32(smem + kSmemV);
+      bool ok = ptx::mbar_wait(&bars[kBarQ], 0, limit);
+
+      auto issue_s = [&](int t, uint32_t kt) {
+#pragma unroll
+        for (int kk = 0; kk < kHeadDim / 16; ++kk)
+          ptx::mma_ss(tmem + col_s(t), desc_kmajor(q_addr[t], kk), desc_kmajor(kt, kk), kIdescS, kk > 0 ? 1u : 0u);
+      };
+      // O_t += P_t(jj) V(jj); returns false if a wait expired
+      auto issue_pv = [&](int t, int jj) -> bool {
+        if (!ptx::mbar_wait(&bars[kBarPFull + t], jj & 1, limit)) return false;
+        if (!ptx::mbar_wait(&bars[kBarVFull + (jj & 1)], (jj >> 1) & 1, limit)) return false;
+        ptx::tc_fence_after();
+        const uint32_t vt = v_addr + (jj & 1) * kTile;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          ptx::mma_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8, desc_v(vt, kk), kIdescPV,
+                      (jj > 0 || kk > 0) ? 1u : 0u);
+        if (t == 1) ptx::mma_commit(&bars[kBarVEmpty + (jj & 1)]);
+        return true;
+      };
+
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        const int s = j & 1;
+        if (!ptx::mbar_wait(&bars[kBarKFull + s], (j >> 1) & 1, limit)) { ok = false; break; }
+        ptx::tc_fence_after();
+        const uint32_t kt = k_addr + s * kTile;
+        issue_s(0, kt);
+        ptx::mma_commit(&bars[kBarSFull + 0]);
+        if (j > 0 && !issue_pv(1, j - 1)) { ok = false; break; }
+        issue_s(1, kt);
+        ptx::mma_commit(&bars[kBarSFull + 1]);
+        ptx::mma_commit(&bars[kBarKEmpty + s]);
+        if (!issue_pv(0, j)) { ok = false; break; }
+      }
+      if (ok && !issue_pv(1, n_tiles - 1)) ok = false;
+      if (ok) ptx::mma_commit(&bars[kBarODone]);
+      if (!ok) atomicOr(p.status, kStatusTimeout);
+      // everything issued must complete before TMEM is released
+      ptx::mma_commit(&bars[kBarDrain]);
+      ptx::mbar_wait(&bars[kBarDrain], 0, kDrainNs);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax warpgroups
+    const int wg = warp >> 2;         // 0 or 1
+    const int wq = warp & 3;          // warp within the warpgroup -> TMEM lanes 32*wq..
+    const int r = threadIdx.x & 127;  // query row within the tile
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const uint32_t tS = lane_base + col_s(wg);
+    const uint32_t tO = lane_base + col_o(wg);
+    const float sl2 = p.scale_log2;
+    float m_used = -INFINITY;
+    float l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_tiles; ++j) {
+      ok = ptx::mbar_wait(&bars[kBarSFull + wg], j & 1, limit);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      ptx::tc_fence_after();
+      int src, krow, vrow, valid;
+      tile_of(p, j, src, krow, vrow, valid);
+      float s[kBN];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t rr[32];
+        ptx::tmem_ld32(tS + 32 * c, rr);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(rr[i]);
+      }
+      if (valid < kBN) {
+#pragma unroll
+        for (int i = 0; i < kBN; ++i)
+          if (i >= valid) s[i] = -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int i = 1; i < kBN; ++i) mx = fmaxf(mx, s[i]);
+      const float m_tile = mx * sl2;
+      const bool need = m_tile > m_used + 8.0f;
+      float alpha = 1.0f;
+      if (need) {
+        alpha = ptx::ex2(m_used - m_tile);
+        m_used = m_tile;
+      }
+      l *= alpha;
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t rr[32];
+          ptx::tmem_ld32(tO + 32 * c, rr);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
+          ptx::tmem_st32(tO + 32 * c, rr);
+        }
+      }
+      float rowsum = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float a = ptx::ex2(fmaf(s[32 * c + 2 * i], sl2, -m_used));
+          const float b = ptx::ex2(fmaf(s[32 * c + 2 * i + 1], sl2, -m_used));
+          rowsum += a + b;
+          pk[i] = pack_bf16x2(a, b);
+        }
+        ptx::tmem_st16(tS + 16 * c, pk);
+      }
+      l += rowsum;
+      ptx::tmem_st_wait();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&bars[kBarPFull + wg]);
+    }
+    if (ok) {
+      ok = ptx::mbar_wait(&bars[kBarODone], 0, limit);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (!ok) {
+      if (lane == 0) atomicOr(p.status, kStatusTimeout);
+    } else {
+      ptx::tc_fence_after();
+      const int row = m0 + wg * kBM + r;
+      const bool live = row < p.Lq;
+      const float inv_l = 1.0f / l;
+      const long long base = (static_cast<long long>(row) * p.H + head) * kHeadDim;
+      FlowStep step;
+      step.sigma = p.sigma;
+      step.renoise = p.sigma_next >= 0.0;
+      step.sigma_next = step.renoise ? p.sigma_next : 0.0;
+      step.one_minus_next = __dsub_rn(1.0, step.sigma_next);
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t rr[32];
+        ptx::tmem_ld32(tO + 32 * c, rr);
+        if (live) {
+          uint32_t ob[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            ob[i] = pack_bf16x2(__uint_as_float(rr[2 * i]) * inv_l, __uint_as_float(rr[2 * i + 1]) * inv_l);
+          uint4* dst = reinterpret_cast<uint4*>(p.out + base + 32 * c);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(ob[4 * v], ob[4 * v + 1], ob[4 * v + 2], ob[4 * v + 3]);
+          if (p.flow) {
+            const uint4* xtp = reinterpret_cast<const uint4*>(p.xt + base + 32 * c);
+            const uint4* ep = reinterpret_cast<const uint4*>(p.eps + base + 32 * c);
+            uint4* x0p = reinterpret_cast<uint4*>(p.x0 + base + 32 * c);
+            uint4* xnp = reinterpret_cast<uint4*>(p.xt_next + base + 32 * c);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const uint4 xv = __ldg(xtp + v);
+              uint4 ev = make_uint4(0, 0, 0, 0);
+              if (step.renoise) ev = __ldg(ep + v);
+              const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+              const uint32_t ew[4] = {ev.x, ev.y, ev.z, ev.w};
+              uint32_t o0[4], o1[4];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const uint32_t vw = ob[4 * v + q];
+                uint16_t a0, a1, b0 = 0, b1 = 0;
+                step.apply(bf16_to_f32(xw[q] & 0xFFFFu), bf16_to_f32(vw & 0xFFFFu), bf16_to_f32(ew[q] & 0xFFFFu), a0, b0);
+                step.apply(bf16_to_f32(xw[q] >> 16), bf16_to_f32(vw >> 16), bf16_to_f32(ew[q] >> 16), a1, b1);
+                o0[q] = static_cast<uint32_t>(a0) | (static_cast<uint32_t>(a1) << 16);
+                o1[q] = static_cast<uint32_t>(b0) | (static_cast<uint32_t>(b1) << 16);
+              }
+              x0p[v] = make_uint4(o0[0], o0[1], o0[2], o0[3]);
+              if (step.renoise) xnp[v] = make_uint4(o1[0], o1[1], o1[2], o1[3]);
+            }
+          }
+        }
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  if (warp == 9) ptx::tmem_dealloc(tmem, 512);
+}
+
+}  // namespace
+
+cudaError_t launch_attention(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_vc,
+                             const CUtensorMap& tm_vn, const AttnParams& p, cudaStream_t stream) {
+  static int configured_device = -1;
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (configured_device != dev) {
+    err = cudaFuncSetAttribute(chunk_attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (err != cudaSuccess) return err;
+    configured_device = dev;
+  }
+  dim3 grid((p.Lq + 2 * kBM - 1) / (2 * kBM), p.H);
+  chunk_attention_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_q, tm_k, tm_vc, tm_vn, p);
+  return cudaGetLastError();
+}
+
+}  // namespace rkv

@@ -60,7 +60,7 @@ def _mix64_np(z: np.ndarray) -> np.ndarray:
     return z ^ (z >> np.uint64(31))
 
 
-def normal_bf16_bits(key: int, start: int, count: int, block: int = 1 << 22) -> np.ndarray:
+def normal_bf16_bits(key: int, start: int, count: int, block: int = 1 << 16) -> np.ndarray:
     """bf16 bit patterns (uint16) of elements ``start .. start+count-1`` of stream ``key``."""
     out = np.empty(count, dtype=np.uint16)
     k = np.uint64(key & MASK64)

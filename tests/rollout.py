@@ -1,0 +1,183 @@
+"""Side-by-side rollout driver for the GPU parity tests: the library (through the
+C ABI) and the oracle run the same chunk schedule on the same seeded inputs.
+
+Inputs: every tensor of every call comes from the ``synth`` generator keyed by
+(seed, config id, layer, chunk, call, tensor tag); the GPU side fills device
+buffers with the CUDA twin, the oracle side draws the same bits with numpy.
+Per chunk: ``reads`` denoise reads (commit=0), then one commit (the t=0 pass).
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import numpy as np
+
+import synth
+from oracle import bf16
+from oracle.layer import OracleLayer
+
+# tolerance of the attention output against the fp64 oracle (bf16 output, N(0,1) inputs)
+MAX_ABS = 1.5e-2
+MEAN_ABS = 1.0e-3
+REL_RMS = 1.0e-2
+
+
+@dataclass
+class Config:
+    name: str
+    cfg_id: int
+    H: int
+    grid_h: int
+    grid_w: int
+    C: int
+    W: int
+    S: int
+    rope_mode: int
+    refs: int = 0          # reference frames written with write_chunk before the chunks (become sinks)
+    chunks: int = 4
+    reads: int = 4
+    layers: int = 1
+    seed: int = 0
+
+    @property
+    def T(self):
+        return self.grid_h * self.grid_w
+
+    @property
+    def Lq(self):
+        return self.C * self.T
+
+
+def key(cfg: Config, layer: int, chunk: int, call: int, tag: str) -> int:
+    return synth.stream_key(cfg.seed, cfg.cfg_id, layer, chunk, call, synth.TAG[tag])
+
+
+def host_bits(cfg, layer, chunk, call, tag, n_tok):
+    return synth.normal_bf16_bits(key(cfg, layer, chunk, call, tag), 0, n_tok * cfg.H * 128).reshape(
+        n_tok, cfg.H, 128)
+
+
+def dev_tensor(torch, cfg, layer, chunk, call, tag, n_tok, out=None):
+    t = out if out is not None else torch.empty((n_tok, cfg.H, 128), dtype=torch.bfloat16, device="cuda")
+    synth.fill_normal_bf16_cuda(t.data_ptr(), t.numel(), key(cfg, layer, chunk, call, tag), 0,
+                                torch.cuda.current_stream().cuda_stream)
+    return t
+
+
+def to_bits(t) -> np.ndarray:
+    import torch
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def compare(out_bits: np.ndarray, ref: np.ndarray):
+    """Error statistics of a bf16 GPU result against the fp64 oracle."""
+    got = bf16.to_f64(out_bits)
+    err = np.abs(got - ref)
+    rms_ref = float(np.sqrt(np.mean(ref ** 2)))
+    rel = float(np.sqrt(np.mean(err ** 2)) / rms_ref) if rms_ref > 0 else 0.0
+    return float(err.max()), float(err.mean()), rel
+
+
+def assert_close(out_bits, ref, what=""):
+    mx, mean, rel = compare(out_bits, ref)
+    assert mx <= MAX_ABS and mean <= MEAN_ABS and rel <= REL_RMS, f"{what}: max {mx:.3e} mean {mean:.3e} rel {rel:.3e}"
+    return mx, mean, rel
+
+
+def cache_logical_bits(lib_h, torch, cfg: Config, layer: int):
+    """The library's raw K/V ring read back in logical (frame) order, token-major [n*T, H, d]."""
+    frames = lib_h.slot_frames(layer)
+    kp, vp = lib_h.cache_ptrs(layer)
+    n_el = cfg.H * cfg.W * cfg.T * 128
+    k_all = _wrap(torch, kp, n_el).view(cfg.H, cfg.W * cfg.T, 128)
+    v_all = _wrap(torch, vp, n_el).view(cfg.H, cfg.W * cfg.T, 128)
+    held = sorted((f, s) for s, f in enumerate(frames) if f >= 0)
+    ks, vs = [], []
+    for f, s in held:
+        ks.append(k_all[:, s * cfg.T:(s + 1) * cfg.T, :].permute(1, 0, 2))
+        vs.append(v_all[:, s * cfg.T:(s + 1) * cfg.T, :].permute(1, 0, 2))
+    if not held:
+        z = np.zeros((0, cfg.H, 128), dtype=np.uint16)
+        return [], z, z
+    return [f for f, _ in held], to_bits(torch.cat(ks)), to_bits(torch.cat(vs))
+
+
+class _CudaArray:
+    def __init__(self, ptr, n):
+        self.__cuda_array_interface__ = {"shape": (n,), "typestr": "<i2", "data": (ptr, False), "version": 3}
+
+
+def _wrap(torch, ptr, n):
+    return torch.as_tensor(_CudaArray(ptr, n), device="cuda").view(torch.bfloat16)
+
+
+@dataclass
+class Rollout:
+    """Drives one config on both sides. ``check(chunk, call)`` decides which calls are compared
+    (returns None to skip, or (rows, heads) to compare those; rows/heads None = all)."""
+    cfg: Config
+    lib: object
+    torch: object
+    oracles: list = field(default_factory=list)
+
+    def __post_init__(self):
+        import rolling_kv_chunked_b200 as rkv
+        c = self.cfg
+        self.h = rkv.RollingKV(c.layers, c.H, 128, c.T, c.W, c.S, c.rope_mode)
+        self.h.set_rope_grid(c.grid_h, c.grid_w, 1.0e4, (22, 21, 21))
+        self.oracles = [OracleLayer(c.H, 128, c.T, c.grid_h, c.grid_w, c.W, c.S, c.rope_mode)
+                        for _ in range(c.layers)]
+        self.f0 = [0] * c.layers
+        if c.refs:
+            for layer in range(c.layers):
+                k = dev_tensor(self.torch, c, layer, -1, 0, "k", c.refs * c.T)
+                v = dev_tensor(self.torch, c, layer, -1, 0, "v", c.refs * c.T)
+                self.h.write_chunk(layer, k, v, c.refs, 0)
+                self.oracles[layer].write_chunk(host_bits(c, layer, -1, 0, "k", c.refs * c.T),
+                                                host_bits(c, layer, -1, 0, "v", c.refs * c.T), c.refs, 0)
+                self.f0[layer] = c.refs
+
+    def run_chunk(self, layer, chunk, check=lambda chunk, call: (None, None), stats=None):
+        c, torch = self.cfg, self.torch
+        f0 = self.f0[layer]
+        out = torch.empty((c.Lq, c.H, 128), dtype=torch.bfloat16, device="cuda")
+        for call in range(c.reads + 1):
+            commit = call == c.reads
+            q = dev_tensor(torch, c, layer, chunk, call, "q", c.Lq)
+            k = dev_tensor(torch, c, layer, chunk, call, "k", c.Lq)
+            v = dev_tensor(torch, c, layer, chunk, call, "v", c.Lq)
+            self.h.chunk_attention(layer, q, k, v, out, c.C, f0, commit)
+            sel = check(chunk, call)
+            orc = self.oracles[layer]
+            if sel is None:
+                if commit:
+                    orc.write_chunk(host_bits(c, layer, chunk, call, "k", c.Lq),
+                                    host_bits(c, layer, chunk, call, "v", c.Lq), c.C, f0)
+                continue
+            rows, heads = sel
+            ref = orc.chunk_attention(host_bits(c, layer, chunk, call, "q", c.Lq),
+                                      host_bits(c, layer, chunk, call, "k", c.Lq),
+                                      host_bits(c, layer, chunk, call, "v", c.Lq), c.C, f0, commit,
+                                      rows=rows, heads=heads)
+            got = to_bits(out)
+            if rows is not None:
+                got = got[np.asarray(rows)]
+            if heads is not None:
+                got = got[:, np.asarray(heads)]
+            r = assert_close(got, ref, f"{c.name} layer {layer} chunk {chunk} call {call}")
+            if stats is not None:
+                stats.append(r)
+        self.f0[layer] = f0 + c.C
+
+    def check_cache(self, layer):
+        c = self.cfg
+        frames, kb, vb = cache_logical_bits(self.h, self.torch, c, layer)
+        orc = self.oracles[layer]
+        assert frames == orc.logical_frames()
+        ok, ov = orc.logical_kv_bits()
+        assert np.array_equal(kb, ok) and np.array_equal(vb, ov)
+        S, R = c.S, c.W - c.S
+        for s, f in enumerate(self.h.slot_frames(layer)):
+            if f >= 0:
+                assert s == (f if f < S else S + (f - S) % R)
+        assert self.h.frames_committed(layer) == self.f0[layer]

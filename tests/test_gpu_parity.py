@@ -1,0 +1,168 @@
+"""GPU parity: the C-ABI kernels against the fp64 oracle on the same seeded inputs.
+
+* the CUDA twin of the input generator reproduces the numpy generator bit for bit;
+* flow x0 / renoise: bit-exact (fp64 arithmetic, no FMA, RNE) incl. a ragged tail;
+* RoPE: every output within one bf16 ulp of the fp64 rotation;
+* chunk attention: every call of small rollouts compared element by element
+  (max |err| <= 1.5e-2, mean |err| <= 1e-3, relative RMS <= 1e-2), cache bytes
+  and slot -> frame map bit-exact after every commit, through warm-up, sink
+  straddling, eviction and ring wrap, several tiles and ragged tails;
+* the fused epilogue equals the standalone epilogue applied to the stored output.
+"""
+import numpy as np
+import pytest
+
+import synth
+from oracle import bf16, flow as oflow
+from oracle.layer import OracleLayer
+from rollout import Config, Rollout, assert_close, dev_tensor, host_bits, to_bits
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("no CUDA device", allow_module_level=True)
+
+import rolling_kv_chunked_b200 as rkv  # noqa: E402
+
+ABS, REL = OracleLayer.ABSOLUTE, OracleLayer.RELATIVE
+
+
+def _dev_bits(key, n):
+    t = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+    synth.fill_normal_bf16_cuda(t.data_ptr(), n, key, 0, torch.cuda.current_stream().cuda_stream)
+    return t
+
+
+def test_generator_twin_bit_exact():
+    for n, k in [(1, 5), (1000003, 11), (4096, synth.stream_key(3, 1, 2))]:
+        got = to_bits(_dev_bits(k, n))
+        assert np.array_equal(got, synth.normal_bf16_bits(k, 0, n))
+    t = torch.empty(777, dtype=torch.bfloat16, device="cuda")
+    synth.fill_normal_bf16_cuda(t.data_ptr(), 777, 9, 12345, torch.cuda.current_stream().cuda_stream)
+    assert np.array_equal(to_bits(t), synth.normal_bf16_bits(9, 12345, 777))
+
+
+@pytest.mark.parametrize("n", [8, 1000003, 2640 * 3072])
+def test_flow_x0_renoise_bit_exact(n):
+    xt, v, eps = (_dev_bits(synth.stream_key(0, 50, i, n % 1000), n) for i in range(3))
+    sig = oflow.sigmas() + [-1.0]
+    for s, sn in zip(sig[:-1], sig[1:]):
+        x0 = torch.empty_like(xt)
+        xn = torch.empty_like(xt)
+        rkv.flow_x0_renoise(xt, v, eps, s, sn, x0, xn if sn >= 0 else None)
+        torch.cuda.synchronize()
+        rx0, rxn = oflow.x0_renoise_bf16(to_bits(xt), to_bits(v), to_bits(eps), s, sn)
+        assert np.array_equal(to_bits(x0), rx0), (n, s)
+        if sn >= 0:
+            assert np.array_equal(to_bits(xn), rxn), (n, s)
+
+
+@pytest.mark.parametrize("mode", [ABS, REL])
+def test_rope_apply_within_one_ulp(mode):
+    H, gh, gw, W, n_frames = 3, 6, 7, 9, 4
+    T = gh * gw
+    h = rkv.RollingKV(1, H, 128, T, W, 2, mode)
+    h.set_rope_grid(gh, gw)
+    orc = OracleLayer(H, 128, T, gh, gw, W, 2, mode)
+    for start, wend in [(0, 4), (5, 9), (37, 41), (200, 300)]:
+        x = _dev_bits(synth.stream_key(1, start), n_frames * T * H * 128).view(n_frames * T, H, 128)
+        xb = to_bits(x)
+        h.rope_apply(x, n_frames, start, wend)
+        torch.cuda.synchronize()
+        ref = orc.rope_apply(xb, n_frames, start, wend)
+        got = bf16.to_f64(to_bits(x))
+        # one bf16 ulp at the reference's magnitude: 2**(floor(log2|ref|) - 7)
+        ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref), 2.0 ** -126))) - 7)
+        assert np.all(np.abs(got - ref) <= ulp), (start, wend)
+    h.close()
+
+
+SMALL = [
+    Config("tiny-abs", 1, H=2, grid_h=4, grid_w=4, C=2, W=6, S=2, rope_mode=ABS, chunks=10),
+    Config("tiny-rel-refs", 2, H=2, grid_h=4, grid_w=4, C=2, W=6, S=2, rope_mode=REL, refs=2, chunks=10),
+    Config("ragged-abs", 3, H=3, grid_h=8, grid_w=10, C=3, W=7, S=2, rope_mode=ABS, chunks=8, reads=2),
+    Config("ragged-rel", 4, H=3, grid_h=8, grid_w=10, C=3, W=7, S=2, rope_mode=REL, refs=1, chunks=8, reads=2),
+    Config("two-cta", 5, H=2, grid_h=10, grid_w=20, C=2, W=5, S=1, rope_mode=ABS, chunks=6, reads=1),
+    Config("straddle", 6, H=2, grid_h=4, grid_w=6, C=4, W=18, S=6, rope_mode=ABS, chunks=8, reads=1),
+    Config("no-sink", 7, H=1, grid_h=3, grid_w=5, C=1, W=4, S=0, rope_mode=REL, chunks=9, reads=1),
+]
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=[c.name for c in SMALL])
+def test_rollout_small_every_call(cfg):
+    ro = Rollout(cfg, rkv, torch)
+    if cfg.refs:
+        ro.check_cache(0)
+    for chunk in range(cfg.chunks):
+        ro.run_chunk(0, chunk)
+        torch.cuda.synchronize()
+        ro.check_cache(0)
+    assert ro.h.poll_device_status() == rkv.OK
+    ro.h.close()
+
+
+def test_fused_flow_epilogue_matches_standalone():
+    cfg = Config("fused", 8, H=2, grid_h=8, grid_w=10, C=3, W=7, S=2, rope_mode=ABS, chunks=1)
+    h = rkv.RollingKV(1, cfg.H, 128, cfg.T, cfg.W, cfg.S, cfg.rope_mode)
+    h.set_rope_grid(cfg.grid_h, cfg.grid_w)
+    Lq, n = cfg.Lq, cfg.Lq * cfg.H * 128
+    q, k, v = (dev_tensor(torch, cfg, 0, 0, 0, t, Lq) for t in ("q", "k", "v"))
+    xt = _dev_bits(synth.stream_key(0, 8, 1), n)
+    eps = _dev_bits(synth.stream_key(0, 8, 2), n)
+    for s, sn in [(1.0, 0.75), (0.25, -1.0)]:
+        out = torch.empty((Lq, cfg.H, 128), dtype=torch.bfloat16, device="cuda")
+        x0 = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+        xn = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+        h.chunk_attention(0, q, k, v, out, cfg.C, 0, False,
+                          flow=dict(xt=xt, eps=eps, sigma=s, sigma_next=sn, x0_out=x0,
+                                    xt_next_out=xn if sn >= 0 else None))
+        torch.cuda.synchronize()
+        rx0, rxn = oflow.x0_renoise_bf16(to_bits(xt), to_bits(out).reshape(-1), to_bits(eps), s, sn)
+        assert np.array_equal(to_bits(x0), rx0)
+        if sn >= 0:
+            assert np.array_equal(to_bits(xn), rxn)
+        # and the attention output itself against the oracle
+        orc = OracleLayer(cfg.H, 128, cfg.T, cfg.grid_h, cfg.grid_w, cfg.W, cfg.S, cfg.rope_mode)
+        ref = orc.chunk_attention(to_bits(q), to_bits(k), to_bits(v), cfg.C, 0, False)
+        assert_close(to_bits(out), ref, "fused")
+    h.close()
+
+
+def test_outputs_are_deterministic():
+    cfg = Config("det", 9, H=2, grid_h=8, grid_w=10, C=3, W=7, S=2, rope_mode=REL, chunks=1)
+    h = rkv.RollingKV(1, cfg.H, 128, cfg.T, cfg.W, cfg.S, cfg.rope_mode)
+    h.set_rope_grid(cfg.grid_h, cfg.grid_w)
+    q, k, v = (dev_tensor(torch, cfg, 0, 0, 0, t, cfg.Lq) for t in ("q", "k", "v"))
+    outs = []
+    for _ in range(3):
+        o = torch.empty((cfg.Lq, cfg.H, 128), dtype=torch.bfloat16, device="cuda")
+        h.chunk_attention(0, q, k, v, o, cfg.C, 0, False)
+        outs.append(to_bits(o))
+    assert np.array_equal(outs[0], outs[1]) and np.array_equal(outs[0], outs[2])
+    h.close()
+
+
+def test_host_errors_launch_nothing():
+    cfg = Config("err", 10, H=2, grid_h=4, grid_w=4, C=2, W=6, S=2, rope_mode=ABS)
+    h = rkv.RollingKV(1, cfg.H, 128, cfg.T, cfg.W, cfg.S, cfg.rope_mode)
+    q, k, v = (dev_tensor(torch, cfg, 0, 0, 0, t, cfg.Lq) for t in ("q", "k", "v"))
+    out = torch.zeros((cfg.Lq, cfg.H, 128), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(rkv.RkvError) as e:
+        h.chunk_attention(0, q, k, v, out, cfg.C, 0, True)          # grid not set yet
+    assert e.value.code == rkv.ERR_STATE
+    h.set_rope_grid(cfg.grid_h, cfg.grid_w)
+    for args, code in [((0, q, k, v, out, cfg.C, 2, False), rkv.ERR_ORDER),
+                       ((0, q, k, v, out, 5, 0, False), rkv.ERR_CAPACITY),
+                       ((1, q, k, v, out, cfg.C, 0, False), rkv.ERR_ARG),
+                       ((0, q, k, v, out, 0, 0, False), rkv.ERR_ARG)]:
+        with pytest.raises(rkv.RkvError) as e:
+            h.chunk_attention(*args)
+        assert e.value.code == code
+    with pytest.raises(rkv.RkvError) as e:
+        h.chunk_attention(0, q.data_ptr() + 2, k, v, out, cfg.C, 0, False)   # misaligned pointer
+    assert e.value.code == rkv.ERR_ARG
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(out).item() == 0
+    assert h.frames_committed(0) == 0 and h.slot_frames(0) == [-1] * cfg.W
+    h.close()
