@@ -235,6 +235,44 @@ def run_rkv(args):
     value = tokens / (ms / 1e3)
 
     # ---- end to end through the C ABI with host buffers (copies inside the timed region)
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, torch, dist, world, stream, pool, outs, x0, step, tokens)
+
+    pk, pk_kind = peaks()
+    mean_kernel_ms = sum(kernel_ms) / max(1, len(kernel_ms))
+    achieved = flops / (sum(kernel_ms) / 1e3) / 1e12 if kernel_ms else None
+    peak = pk["bf16_tflops_sustained"]
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": cfg["workload"], "queries_per_call": Lq, "keys_per_call": W * T,
+                   "calls_per_step": 5, "parallelism": f"replicas x{world} (no data-path collective)",
+                   "l2": f"inputs larger than L2 ({(15 * Lq * H * 128 + 4 * Lq * H * 128) * 2 / 1e6:.0f} MB per step)"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": (achieved / peak) if achieved else None, "traffic": None,
+                     "kernel": "chunk_attention_kernel", "peak_source": f"{pk_kind} bf16_tflops_sustained",
+                     "frac_of_burst": (achieved / pk["bf16_tflops"]) if achieved else None,
+                     "mean_kernel_ms": mean_kernel_ms, "launches_timed": len(kernel_ms),
+                     "flops_per_launch": flops / max(1, 5 * args.steps)},
+        "e2e": e2e,
+        "gpu_launches": 11 * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(cfg, budget_s=args.cpu_seconds)
+    h.close()
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+def run_e2e(args, torch, dist, world, stream, pool, outs, x0, step, tokens):
+    """Same steps through the public API with the inputs in pinned host memory: each step copies
+    its inputs host->device and its results (five attention outputs, final x0) device->host."""
+    Lq, H = outs[0].shape[0], outs[0].shape[1]
     hostset = []
     for i in range(2):
         src = pool[i]
@@ -276,35 +314,7 @@ def run_rkv(args):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e_ms = float(t.item())
     e2e_value = tokens / (e2e_ms / 1e3)
-
-    pk, pk_kind = peaks()
-    mean_kernel_ms = sum(kernel_ms) / max(1, len(kernel_ms))
-    achieved = flops / (sum(kernel_ms) / 1e3) / 1e12 if kernel_ms else None
-    peak = pk["bf16_tflops_sustained"]
-    result = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": cfg["workload"], "queries_per_call": Lq, "keys_per_call": W * T,
-                   "calls_per_step": 5, "parallelism": f"replicas x{world} (no data-path collective)",
-                   "l2": f"inputs larger than L2 ({(15 * Lq * H * 128 + 4 * Lq * H * 128) * 2 / 1e6:.0f} MB per step)"},
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": (achieved / peak) if achieved else None, "traffic": None,
-                     "kernel": "chunk_attention_kernel", "peak_source": f"{pk_kind} bf16_tflops_sustained",
-                     "frac_of_burst": (achieved / pk["bf16_tflops"]) if achieved else None,
-                     "mean_kernel_ms": mean_kernel_ms, "launches_timed": len(kernel_ms),
-                     "flops_per_launch": flops / max(1, 5 * args.steps)},
-        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 11 * args.steps,
-        "clocks": clk,
-    }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(cfg, budget_s=args.cpu_seconds)
-    h.close()
-    if world > 1:
-        dist.destroy_process_group()
-    if rank == 0:
-        print(json.dumps(result), flush=True)
+    return {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
 
 # ---------------------------------------------------------------------- oracle arm
@@ -391,6 +401,7 @@ def main():
     ap.add_argument("--impl", default="rkv", choices=["rkv", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end pass")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
