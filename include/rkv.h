@@ -180,6 +180,36 @@ int rkv_poll_device_status(rkv_handle h, void* stream);
  *  wait expire so the timeout path can be tested. Errors: RKV_ERR_ARG. */
 int rkv_set_wait_limit(rkv_handle h, long long nanoseconds);
 
+/*
+ * rkv_chunk_attention_noalloc - chunk attention without a handle and without
+ *  allocating device memory, for callers that may not call cudaMalloc (a host
+ *  framework whose allocator must own every byte, a real-time or sandboxed
+ *  process that forbids allocation after start-up, a library limited to the
+ *  buffers its caller passes in). The pages have no counterpart: this is an
+ *  interface for such callers, not a step of the method.
+ *  The caller holds the window itself: k_window / v_window are the
+ *  n_window_frames frames the chunk attends to, in logical order (sinks,
+ *  history, then the chunk's own n_frames frames last), token-major
+ *  [n_window_frames*T, H, 128] bf16; frame_ids (host, n_window_frames ints) are
+ *  their absolute frame indices, the last n_frames being start_frame.. .
+ *  q and out are [n_frames*T, H, 128]. RoPE: theta 1e4, pairs 22/21/21, time id
+ *  the frame index (RKV_ROPE_ABSOLUTE, ids < 4096) or re-based and clamped to
+ *  [0, window_frames-1] (RKV_ROPE_RELATIVE). Output as rkv_chunk_attention.
+ *  Scratch: one static device array of 32 MiB per device (RoPE tables, rotated
+ *  Q and K, a status word), held from the library's first use on that device
+ *  until exit. The first call on a device looks up the array's device address;
+ *  make that first call before any stream capture. Calls share the array: calls
+ *  that overlap on the GPU race. An expired device wait is not reported here.
+ *  Errors: RKV_ERR_ARG, RKV_ERR_UNSUPPORTED (absolute id >= 4096, window in more
+ *  than 7 runs of consecutive frames), RKV_ERR_CAPACITY (the window, queries and
+ *  tables need more than the 32 MiB array), RKV_ERR_CUDA. Argument and size
+ *  errors launch nothing.
+ */
+int rkv_chunk_attention_noalloc(const void* q, const void* k_window, const void* v_window, void* out,
+                                int H, int tokens_per_frame, int grid_h, int grid_w, int window_frames,
+                                int rope_mode, int n_frames, int start_frame, const int* frame_ids,
+                                int n_window_frames, void* stream);
+
 /* rkv_timing_begin - start recording a CUDA event pair around each attention
  *  kernel launch (on the caller's stream), for at most max_launches launches.
  *  Instrumentation only: nothing is skipped. Errors: RKV_ERR_ARG, RKV_ERR_CUDA. */

@@ -60,6 +60,7 @@ _SIGS = {
     "rkv_status_string": ([_c_int], ctypes.c_char_p),
     "rkv_poll_device_status": ([_vp, _vp], _c_int),
     "rkv_set_wait_limit": ([_vp, _c_ll], _c_int),
+    "rkv_chunk_attention_noalloc": ([_vp, _vp, _vp, _vp] + [_c_int] * 8 + [_int_p, _c_int, _vp], _c_int),
     "rkv_timing_begin": ([_vp, _c_int], _c_int),
     "rkv_timing_end": ([_vp, ctypes.POINTER(ctypes.c_float), _c_int, _int_p], _c_int),
     "rkv_plan_window": ([_c_int, _c_int, _c_int, _c_int, _c_int, _int_p, _c_int, _int_p], _c_int),

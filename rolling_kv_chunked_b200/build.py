@@ -25,7 +25,7 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 LIB = os.path.join(HERE, "librkv.so")
 SYNTH_LIB = os.path.join(ROOT, "synth", "libsynth.so")
 
-CU_SOURCES = ["rkv_kernels.cu", "rkv_attention.cu"]
+CU_SOURCES = ["rkv_kernels.cu", "rkv_attention.cu", "rkv_noalloc.cu"]
 CPP_SOURCES = ["rkv_host.cpp"]
 HEADERS = ["ptx_sm100.cuh", "numeric.cuh", "rkv_internal.h"]
 
