@@ -25,7 +25,11 @@
 //   S0(j) = Q0 K_j^T, PV1(j-1), S1(j) = Q1 K_j^T, PV0(j)
 // so that while one softmax warpgroup works on its tile the tensor core runs the
 // other tile's products. Online softmax in the log2 domain with a lazy rescale
-// (O is rescaled only when a row maximum grows by more than 2^8).
+// (O is rescaled only when a row maximum grows by more than 2^8). Each softmax thread
+// reads its S row twice from TMEM (once for the maximum, then 64 columns at a time for
+// the exponentials), which keeps the warpgroups within their register budget without
+// spills; exponentials run on the special-function unit, one pair in eight on the FMA
+// pipe as a polynomial, and P is rounded to bf16 with integer operations.
 //
 // Every mbarrier wait is bounded in wall time; on expiry the kernel records
 // kStatusTimeout in the status word, stops issuing work, waits (bounded) for the
@@ -103,8 +107,67 @@ __device__ __forceinline__ uint64_t desc_v(uint32_t tile_addr, int kk) {
   return ptx::smem_desc_sw128(tile_addr + kk * 2048, kSlab, 1024);
 }
 
+// two fp32 -> packed bf16x2 (lo in the low half), round to nearest even, one conversion
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  return static_cast<uint32_t>(f32_to_bf16_rne(lo)) | (static_cast<uint32_t>(f32_to_bf16_rne(hi)) << 16);
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// 2^x for two lanes on the FMA / integer pipes instead of the special-function unit:
+// t = x + 1.5*2^23 rounds x to the nearest integer r (kept in t's low mantissa bits),
+// f = x - r in [-1/2, 1/2], 2^f by a degree-3 polynomial (max relative error 7.5e-5,
+// coefficients fitted for minimal relative error by rolling_kv_chunked_b200/exp2_poly.py),
+// then r is added to the exponent field (the bits of 1.5*2^23 vanish under << 23).
+// x is clamped at -125 so the result stays a positive normal number.
+__device__ __forceinline__ void exp2_poly_x2(uint64_t x2, float& y0, float& y1) {
+  float x0, x1;
+  ptx::f2_unpack(x2, x0, x1);
+  const uint64_t x = ptx::f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+  const uint64_t magic = ptx::f2_pack(12582912.0f, 12582912.0f);
+  const uint64_t neg_magic = ptx::f2_pack(-12582912.0f, -12582912.0f);
+  const uint64_t neg_one = ptx::f2_pack(-1.0f, -1.0f);
+  const uint64_t t = ptx::f2_add(x, magic);
+  const uint64_t r = ptx::f2_add(t, neg_magic);
+  const uint64_t f = ptx::f2_fma(r, neg_one, x);
+  uint64_t q = ptx::f2_fma(ptx::f2_pack(0.05517166493030145f, 0.05517166493030145f), f,
+                           ptx::f2_pack(0.24261112187715117f, 0.24261112187715117f));
+  q = ptx::f2_fma(q, f, ptx::f2_pack(0.6932609862225388f, 0.6932609862225388f));
+  q = ptx::f2_fma(q, f, ptx::f2_pack(0.9999280735783096f, 0.9999280735783096f));
+  float t0, t1, q0, q1;
+  ptx::f2_unpack(t, t0, t1);
+  ptx::f2_unpack(q, q0, q1);
+  y0 = __uint_as_float((__float_as_uint(t0) << 23) + __float_as_uint(q0));
+  y1 = __uint_as_float((__float_as_uint(t1) << 23) + __float_as_uint(q1));
+}
+
+// Softmax numerators of 64 keys (one half of a 128-key row): p = 2^(s * sl2 - m), rounded to
+// bf16 on the integer ALU (add half an ulp, keep the upper halves) and packed in pairs into
+// 32 TMEM columns at tP; row sums accumulate in acc.
+// kPoly: kPolyPairs of every 8 pairs take the polynomial path (full tiles only).
+#ifndef RKV_POLY_PAIRS
+#define RKV_POLY_PAIRS 1
+#endif
+constexpr int kPolyPairs = RKV_POLY_PAIRS;
+template <bool kPoly>
+__device__ __forceinline__ void softmax_half(const uint32_t* sh, uint64_t c2, uint64_t nm2, uint32_t tP,
+                                             uint64_t (&acc)[4]) {
+  uint32_t pk[kBN / 4];
+#pragma unroll
+  for (int k = 0; k < kBN / 4; ++k) {
+    const uint64_t x = ptx::f2_fma(ptx::f2_pack(__uint_as_float(sh[2 * k]), __uint_as_float(sh[2 * k + 1])), c2, nm2);
+    float a, b;
+    if (kPoly && (k & 7) < kPolyPairs) {
+      exp2_poly_x2(x, a, b);
+    } else {
+      float x0, x1;
+      ptx::f2_unpack(x, x0, x1);
+      a = ptx::ex2(x0);
+      b = ptx::ex2(x1);
+    }
+    acc[k & 3] = ptx::f2_add(acc[k & 3], ptx::f2_pack(a, b));
+    pk[k] = __byte_perm(__float_as_uint(a) + 0x8000u, __float_as_uint(b) + 0x8000u, 0x7632);
+  }
+  ptx::tmem_st32(tP, pk);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -252,23 +315,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::tc_fence_after();
       int src, krow, vrow, valid;
       tile_of(p, j, src, krow, vrow, valid);
-      float s[kBN];
+      float m_tile;
+      {
+        // pass 1: the row maximum only
+        uint32_t sr[kBN];
+        ptx::tmem_ld128(tS, sr);
+        if (valid < kBN) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t rr[32];
-        ptx::tmem_ld32(tS + 32 * c, rr);
+          for (int i = 0; i < kBN; ++i)
+            if (i >= valid) sr[i] = 0xff800000u;
+        }
+        float mq[4];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(rr[i]);
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t* t = sr + 32 * c;
+          float m = ptx::fmax3(__uint_as_float(t[0]), __uint_as_float(t[1]), __uint_as_float(t[2]));
+#pragma unroll
+          for (int i = 3; i < 31; i += 2) m = ptx::fmax3(m, __uint_as_float(t[i]), __uint_as_float(t[i + 1]));
+          mq[c] = fmaxf(m, __uint_as_float(t[31]));
+        }
+        m_tile = ptx::fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3])) * sl2;
       }
-      if (valid < kBN) {
-#pragma unroll
-        for (int i = 0; i < kBN; ++i)
-          if (i >= valid) s[i] = -INFINITY;
-      }
-      float mx = s[0];
-#pragma unroll
-      for (int i = 1; i < kBN; ++i) mx = fmaxf(mx, s[i]);
-      const float m_tile = mx * sl2;
       const bool need = m_tile > m_used + 8.0f;
       float alpha = 1.0f;
       if (need) {
@@ -286,20 +353,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           ptx::tmem_st32(tO + 32 * c, rr);
         }
       }
-      float rowsum = 0.f;
+      // p = 2^(s * scale_log2 - m_used), two lanes per instruction
+      const uint64_t c2 = ptx::f2_pack(sl2, sl2);
+      const uint64_t nm2 = ptx::f2_pack(-m_used, -m_used);
+      uint64_t acc[4] = {0, 0, 0, 0};
+      // pass 2: reload 64 columns at a time; P of the first half overwrites S columns
+      // 0..31, already read, the second half's loads touch columns 64..127 only
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t sh[kBN / 2];
+        ptx::tmem_ld64(tS + 64 * hh, sh);
+        if (valid < kBN) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float a = ptx::ex2(fmaf(s[32 * c + 2 * i], sl2, -m_used));
-          const float b = ptx::ex2(fmaf(s[32 * c + 2 * i + 1], sl2, -m_used));
-          rowsum += a + b;
-          pk[i] = pack_bf16x2(a, b);
+          for (int i = 0; i < kBN / 2; ++i)
+            if (64 * hh + i >= valid) sh[i] = 0xff800000u;
+          softmax_half<false>(sh, c2, nm2, tS + 32 * hh, acc);
+        } else {
+          softmax_half<true>(sh, c2, nm2, tS + 32 * hh, acc);
         }
-        ptx::tmem_st16(tS + 16 * c, pk);
       }
-      l += rowsum;
+      float rs[8];
+      ptx::f2_unpack(ptx::f2_add(acc[0], acc[1]), rs[0], rs[1]);
+      ptx::f2_unpack(ptx::f2_add(acc[2], acc[3]), rs[2], rs[3]);
+      l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
       ptx::tmem_st_wait();
       ptx::tc_fence_before();
       ptx::mbar_arrive(&bars[kBarPFull + wg]);
