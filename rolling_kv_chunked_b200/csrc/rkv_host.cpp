@@ -104,14 +104,14 @@ bool encode_map(CUtensorMap* m, const void* base, uint64_t dim1, uint64_t dim2, 
   return r == CUDA_SUCCESS;
 }
 
-// head-major [H][rows][d]
-bool encode_head_major(CUtensorMap* m, const void* base, int rows, int H) {
-  return encode_map(m, base, rows, H, kHeadDim * 2, static_cast<uint64_t>(rows) * kHeadDim * 2, 128, 1);
+// head-major [H][rows][d], boxes of box_rows rows of one head
+bool encode_head_major(CUtensorMap* m, const void* base, int rows, int H, int box_rows) {
+  return encode_map(m, base, rows, H, kHeadDim * 2, static_cast<uint64_t>(rows) * kHeadDim * 2, box_rows, 1);
 }
 
-// token-major [rows][H][d]
-bool encode_token_major(CUtensorMap* m, const void* base, int rows, int H) {
-  return encode_map(m, base, H, rows, kHeadDim * 2, static_cast<uint64_t>(H) * kHeadDim * 2, 1, 128);
+// token-major [rows][H][d], boxes of box_rows tokens of one head
+bool encode_token_major(CUtensorMap* m, const void* base, int rows, int H, int box_rows) {
+  return encode_map(m, base, H, rows, kHeadDim * 2, static_cast<uint64_t>(H) * kHeadDim * 2, 1, box_rows);
 }
 
 bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -302,9 +302,9 @@ RKV_API int rkv_create(int layers, int H, int d, int tokens_per_frame, int windo
       rc = RKV_ERR_CUDA;
       break;
     }
-    if (!encode_head_major(&L.tm_q, L.qstage, static_cast<int>(q_rows), H) ||
-        !encode_head_major(&L.tm_k, L.rotk, static_cast<int>(rot_rows), H) ||
-        !encode_head_major(&L.tm_vc, L.v, static_cast<int>(ring_rows), H)) {
+    if (!encode_head_major(&L.tm_q, L.qstage, static_cast<int>(q_rows), H, rkv::kQueryBox) ||
+        !encode_head_major(&L.tm_k, L.rotk, static_cast<int>(rot_rows), H, rkv::kKeyBox) ||
+        !encode_head_major(&L.tm_vc, L.v, static_cast<int>(ring_rows), H, rkv::kKeyBox)) {
       rc = RKV_ERR_CUDA;
       break;
     }
@@ -490,7 +490,7 @@ RKV_API int rkv_chunk_attention_flow(rkv_handle h, int layer, const void* q, con
       s.k_row0 = static_cast<int>(ring_rows);
       s.v_row0 = 0;
     }
-    ap.n_tiles += (s.n_rows + 127) / 128;
+    ap.n_tiles += (s.n_rows + rkv::kKeyBox - 1) / rkv::kKeyBox;
   }
   ap.H = h->H;
   ap.Lq = C * T;
@@ -510,7 +510,7 @@ RKV_API int rkv_chunk_attention_flow(rkv_handle h, int layer, const void* q, con
   ap.status = h->status;
   ap.wait_limit_ns = h->wait_ns;
   CUtensorMap tm_vn;
-  if (!encode_token_major(&tm_vn, v, C * T, h->H)) return RKV_ERR_CUDA;
+  if (!encode_token_major(&tm_vn, v, C * T, h->H, rkv::kKeyBox)) return RKV_ERR_CUDA;
   const bool timed = h->timing && h->timing_n < h->timing_max;
   if (timed && cudaEventRecord(h->ev_start[h->timing_n], st) != cudaSuccess) return RKV_ERR_CUDA;
   rc = cuda_rc(rkv::launch_attention(L.tm_q, L.tm_k, L.tm_vc, tm_vn, ap, st));

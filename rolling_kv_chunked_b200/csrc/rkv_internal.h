@@ -9,6 +9,10 @@
 namespace rkv {
 
 constexpr int kHeadDim = 128;
+// TMA box heights of the attention kernel's tensor maps: queries are loaded in
+// 128-row tiles, keys and values in 128-row tiles.
+constexpr int kQueryBox = 128;
+constexpr int kKeyBox = 128;
 constexpr int kMaxRuns = 8;
 constexpr int kMaxSegs = 4;
 constexpr int kTimeTable = 65536;  // time ids in [0, kTimeTable) have cos/sin rows
@@ -61,6 +65,7 @@ cudaError_t launch_flow(const FlowParams& p, cudaStream_t stream);
 // ---------------------------------------------------------------- attention
 // One key segment: K rows [k_row0, k_row0 + n_rows) of the rotated-K buffer and
 // V rows [v_row0, ...) of either the cache V ring (src 0) or the caller's v (src 1).
+// tm_q must use boxes of kQueryBox rows; tm_k, tm_vc and tm_vn boxes of kKeyBox rows.
 struct AttnSeg {
   int src;
   int k_row0;
@@ -71,7 +76,7 @@ struct AttnSeg {
 struct AttnParams {
   AttnSeg seg[kMaxSegs];
   int n_segs;
-  int n_tiles;  // sum over segments of ceil(n_rows / 128)
+  int n_tiles;  // sum over segments of ceil(n_rows / kKeyBox)
   int H, Lq;
   float scale_log2;  // log2(e) / sqrt(d)
   uint16_t* out;     // [Lq, H, d]

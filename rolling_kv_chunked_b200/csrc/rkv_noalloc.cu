@@ -203,9 +203,9 @@ extern "C" __attribute__((visibility("default"))) int rkv_chunk_attention_noallo
   if (rc != RKV_OK) return rc;
 
   CUtensorMap tm_q, tm_k, tm_v;
-  if (!encode(&tm_q, qs, Lq, H, kHeadDim * 2, Lq * kHeadDim * 2, 128, 1) ||
-      !encode(&tm_k, ks, Lk, H, kHeadDim * 2, Lk * kHeadDim * 2, 128, 1) ||
-      !encode(&tm_v, v_window, H, Lk, kHeadDim * 2, static_cast<uint64_t>(H) * kHeadDim * 2, 1, 128))
+  if (!encode(&tm_q, qs, Lq, H, kHeadDim * 2, Lq * kHeadDim * 2, kQueryBox, 1) ||
+      !encode(&tm_k, ks, Lk, H, kHeadDim * 2, Lk * kHeadDim * 2, kKeyBox, 1) ||
+      !encode(&tm_v, v_window, H, Lk, kHeadDim * 2, static_cast<uint64_t>(H) * kHeadDim * 2, 1, kKeyBox))
     return RKV_ERR_CUDA;
   AttnParams ap;
   std::memset(&ap, 0, sizeof(ap));
@@ -214,7 +214,7 @@ extern "C" __attribute__((visibility("default"))) int rkv_chunk_attention_noallo
   ap.seg[0].k_row0 = 0;
   ap.seg[0].v_row0 = 0;
   ap.seg[0].n_rows = static_cast<int>(Lk);
-  ap.n_tiles = static_cast<int>((Lk + 127) / 128);
+  ap.n_tiles = static_cast<int>((Lk + kKeyBox - 1) / kKeyBox);
   ap.H = H;
   ap.Lq = static_cast<int>(Lq);
   ap.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(kHeadDim)));
