@@ -50,6 +50,25 @@ SIGMAS = [1.0, 0.75, 0.5, 0.25]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+ATTN_SRC = os.path.join(ROOT, "rolling_kv_chunked_b200", "csrc", "rkv_attention.cu")
+
+
+def profiled_traffic(config_name):
+    """DRAM bytes per attention launch from the committed ncu record of this workload, if that
+    record was taken on the current kernel source (same sha256), else None."""
+    import hashlib
+    rec = os.path.join(ROOT, "profiles", f"chunk_attention_{config_name}.traffic.json")
+    if not os.path.exists(rec):
+        return None, None
+    with open(rec) as fh:
+        r = json.load(fh)
+    with open(ATTN_SRC, "rb") as fh:
+        sha = hashlib.sha256(fh.read()).hexdigest()
+    if r.get("kernel_source_sha256") != sha:
+        return None, "kernel changed since the counters were taken"
+    return r["dram_bytes_per_launch"], rec
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -164,18 +183,22 @@ def run_rkv(args):
     xn = [torch.empty((Lq, H * 128), **bf) for _ in range(2)]
     state = {"f0": 0}
 
-    def step(inp):
+    def step(inp, o=None, x0_buf=None, st=None):
+        """One chunk: four denoise reads with the fused x0 / renoise epilogue, then the commit."""
+        o = outs if o is None else o
+        x0_buf = x0 if x0_buf is None else x0_buf
+        st = sp if st is None else st
         f0 = state["f0"]
         xt = inp["xt"]
         for s in range(4):
             sn = SIGMAS[s + 1] if s < 3 else -1.0
             nxt = xn[s % 2] if sn >= 0 else None
-            h.chunk_attention(0, inp["q"][s], inp["k"][s], inp["v"][s], outs[s], C, f0, False, stream=sp,
+            h.chunk_attention(0, inp["q"][s], inp["k"][s], inp["v"][s], o[s], C, f0, False, stream=st,
                               flow=dict(xt=xt, eps=inp["eps"][s] if sn >= 0 else None, sigma=SIGMAS[s],
-                                        sigma_next=sn, x0_out=x0, xt_next_out=nxt))
+                                        sigma_next=sn, x0_out=x0_buf, xt_next_out=nxt))
             if nxt is not None:
                 xt = nxt
-        h.chunk_attention(0, inp["q"][4], inp["k"][4], inp["v"][4], outs[4], C, f0, True, stream=sp)
+        h.chunk_attention(0, inp["q"][4], inp["k"][4], inp["v"][4], o[4], C, f0, True, stream=st)
         state["f0"] = f0 + C
 
     # reference frames (sinks) and roll the window to steady state
@@ -237,9 +260,11 @@ def run_rkv(args):
     # ---- end to end through the C ABI with host buffers (copies inside the timed region)
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, torch, dist, world, stream, pool, outs, x0, step, tokens)
+        e2e = run_e2e(args, torch, dist, world, pool, step, tokens)
+    hbm = None if args.no_hbm else measure_hbm_kernels(torch, rkv, synth, cfg, rank)
 
     pk, pk_kind = peaks()
+    traffic, traffic_src = profiled_traffic(args.config)
     mean_kernel_ms = sum(kernel_ms) / max(1, len(kernel_ms))
     achieved = flops / (sum(kernel_ms) / 1e3) / 1e12 if kernel_ms else None
     peak = pk["bf16_tflops_sustained"]
@@ -251,12 +276,14 @@ def run_rkv(args):
                    "calls_per_step": 5, "parallelism": f"replicas x{world} (no data-path collective)",
                    "l2": f"inputs larger than L2 ({(15 * Lq * H * 128 + 4 * Lq * H * 128) * 2 / 1e6:.0f} MB per step)"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": (achieved / peak) if achieved else None, "traffic": None,
+                     "frac": (achieved / peak) if achieved else None, "traffic": traffic,
+                     "traffic_source": traffic_src,
                      "kernel": "chunk_attention_kernel", "peak_source": f"{pk_kind} bf16_tflops_sustained",
                      "frac_of_burst": (achieved / pk["bf16_tflops"]) if achieved else None,
                      "mean_kernel_ms": mean_kernel_ms, "launches_timed": len(kernel_ms),
                      "flops_per_launch": flops / max(1, 5 * args.steps)},
         "e2e": e2e,
+        "hbm_kernels": hbm,
         "gpu_launches": 11 * args.steps,
         "clocks": clk,
     }
@@ -269,52 +296,142 @@ def run_rkv(args):
         print(json.dumps(result), flush=True)
 
 
-def run_e2e(args, torch, dist, world, stream, pool, outs, x0, step, tokens):
-    """Same steps through the public API with the inputs in pinned host memory: each step copies
-    its inputs host->device and its results (five attention outputs, final x0) device->host."""
-    Lq, H = outs[0].shape[0], outs[0].shape[1]
-    hostset = []
+def run_e2e(args, torch, dist, world, pool, step, tokens):
+    """The same steps through the public API with every input in pinned host memory: each
+    step copies its inputs host -> device and its results (the five attention outputs and
+    the final x0) device -> host. Copies run on their own streams, double-buffered, so the
+    transfers of one step overlap the kernels of the previous one."""
+    Lq, H = pool[0]["q"][0].shape[0], pool[0]["q"][0].shape[1]
+    bf = dict(dtype=torch.bfloat16, device="cuda")
+    comp = torch.cuda.Stream()
+    h2d_s = torch.cuda.Stream()
+    d2h_s = torch.cuda.Stream()
+    host_in = []
     for i in range(2):
-        src = pool[i]
-        hostset.append({k: ([t.cpu().pin_memory() for t in v] if isinstance(v, list) else v.cpu().pin_memory())
-                        for k, v in src.items()})
-    dev = pool[0]
-    host_out = [torch.empty((Lq, H, 128), dtype=torch.bfloat16).pin_memory() for _ in range(5)]
-    host_x0 = torch.empty((Lq, H * 128), dtype=torch.bfloat16).pin_memory()
-    h2d = sum(t.numel() * 2 for k, v in hostset[0].items() for t in (v if isinstance(v, list) else [v]))
-    d2h = sum(t.numel() * 2 for t in host_out) + host_x0.numel() * 2
+        host_in.append({k: ([t.cpu().pin_memory() for t in v] if isinstance(v, list) else v.cpu().pin_memory())
+                        for k, v in pool[i].items()})
+    dev_in = pool                                            # two device input sets
+    dev_out = [[torch.empty((Lq, H, 128), **bf) for _ in range(5)] for _ in range(2)]
+    dev_x0 = [torch.empty((Lq, H * 128), **bf) for _ in range(2)]
+    host_out = [[torch.empty((Lq, H, 128), dtype=torch.bfloat16).pin_memory() for _ in range(5)] for _ in range(2)]
+    host_x0 = [torch.empty((Lq, H * 128), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    h2d = sum(t.numel() * 2 for v in host_in[0].values() for t in (v if isinstance(v, list) else [v]))
+    d2h = sum(t.numel() * 2 for t in host_out[0]) + host_x0[0].numel() * 2
+    ev_in = [torch.cuda.Event() for _ in range(2)]      # inputs of set b landed
+    ev_done = [torch.cuda.Event() for _ in range(2)]    # kernels of set b finished
+    ev_out = [torch.cuda.Event() for _ in range(2)]     # results of set b copied out
 
-    def e2e_step(i):
-        hs = hostset[i % 2]
-        for key_, val in hs.items():
+    def copy_set(dst, src):
+        for key_, val in src.items():
             if isinstance(val, list):
-                for d_, s_ in zip(dev[key_], val):
+                for d_, s_ in zip(dst[key_], val):
                     d_.copy_(s_, non_blocking=True)
             else:
-                dev[key_].copy_(val, non_blocking=True)
-        step(dev)
-        for d_, s_ in zip(host_out, outs):
-            d_.copy_(s_, non_blocking=True)
-        host_x0.copy_(x0, non_blocking=True)
+                dst[key_].copy_(val, non_blocking=True)
 
-    e2e_step(0)
+    def run(n):
+        for i in range(n):
+            b = i % 2
+            with torch.cuda.stream(h2d_s):
+                if i >= 2:
+                    h2d_s.wait_event(ev_done[b])           # set b's inputs are free again
+                copy_set(dev_in[b], host_in[b])
+                ev_in[b].record(h2d_s)
+            comp.wait_event(ev_in[b])
+            if i >= 2:
+                comp.wait_event(ev_out[b])                 # set b's outputs were copied out
+            step(dev_in[b], dev_out[b], dev_x0[b], comp.cuda_stream)
+            ev_done[b].record(comp)
+            with torch.cuda.stream(d2h_s):
+                d2h_s.wait_event(ev_done[b])
+                for d_, s_ in zip(host_out[b], dev_out[b]):
+                    d_.copy_(s_, non_blocking=True)
+                host_x0[b].copy_(dev_x0[b], non_blocking=True)
+                ev_out[b].record(d2h_s)
+
+    run(2)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(args.steps):
-        e2e_step(i)
-    e1.record(stream)
+    e0.record(comp)
+    h2d_s.wait_event(e0)
+    run(args.steps)
+    comp.wait_stream(h2d_s)
+    comp.wait_stream(d2h_s)
+    e1.record(comp)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
     if world > 1:
         t = torch.tensor([e2e_ms], device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e_ms = float(t.item())
-    e2e_value = tokens / (e2e_ms / 1e3)
-    return {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    return {"value": tokens / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": e2e_ms / args.steps, "overlap": "h2d / kernels / d2h on three streams, double-buffered"}
+
+
+def measure_hbm_kernels(torch, rkv, synth, cfg, rank, reps=20):
+    """Achieved HBM bandwidth of the memory-bound kernels at the workload's sizes, timed with
+    CUDA events on their stream; every launch touches a different buffer set and the sets
+    together exceed the 126 MB L2, so each launch streams from HBM."""
+    H, C, W, S = cfg["H"], cfg["C"], cfg["W"], cfg["S"]
+    T = cfg["gh"] * cfg["gw"]
+    Lq = C * T
+    n = Lq * H * 128
+    st = torch.cuda.current_stream()
+    sp = st.cuda_stream
+    bf = dict(dtype=torch.bfloat16, device="cuda")
+    n_sets = max(2, -(-int(320e6) // (n * 2 * 5)))       # >= 320 MB cycled
+
+    def fill(t, *f):
+        synth.fill_normal_bf16_cuda(t.data_ptr(), t.numel(), synth.stream_key(rank, 88, *f), 0, sp)
+        return t
+
+    def timed(fn):
+        fn(0)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        for i in range(reps):
+            fn(i)
+        e1.record(st)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps / 1e3
+
+    res = {}
+    # K4: x0 = xt - sigma v; xt' = (1 - sigma') x0 + sigma' eps; 3 reads + 2 writes of bf16
+    sets = [[fill(torch.empty(n, **bf), i, j) for j in range(5)] for i in range(n_sets)]
+    sec = timed(lambda i: rkv.flow_x0_renoise(sets[i % n_sets][0], sets[i % n_sets][1], sets[i % n_sets][2],
+                                              1.0, 0.75, sets[i % n_sets][3], sets[i % n_sets][4], stream=sp))
+    res["flow_x0_renoise"] = {"bytes_per_launch": 10 * n, "GB/s": 10 * n / sec / 1e9}
+    del sets
+    # K3: in-place RoPE of a [Lq, H, 128] tensor, one read + one write
+    bufs = [fill(torch.empty((Lq, H, 128), **bf), 50, i) for i in range(2 * n_sets)]
+    hr = rkv.RollingKV(1, H, 128, T, W, S, cfg["mode"])
+    hr.set_rope_grid(cfg["gh"], cfg["gw"])
+    sec = timed(lambda i: hr.rope_apply(bufs[i % len(bufs)], C, 0, C, stream=sp))
+    res["rope_apply"] = {"bytes_per_launch": 4 * n, "GB/s": 4 * n / sec / 1e9}
+    # K1: the ring write-back (rkv_write_chunk): K and V read and written once; in absolute
+    # mode the rotated copy of K is written as well
+    hw = rkv.RollingKV(1, H, 128, T, W, S, cfg["mode"])
+    hw.set_rope_grid(cfg["gh"], cfg["gw"])
+    state = {"f": 0}
+
+    def write(i):
+        hw.write_chunk(0, bufs[(2 * i) % len(bufs)], bufs[(2 * i + 1) % len(bufs)], C, state["f"], stream=sp)
+        state["f"] += C
+    sec = timed(write)
+    per = 8 * n + (4 * n if cfg["mode"] == 0 else 0)
+    res["commit_write"] = {"bytes_per_launch": per, "GB/s": per / sec / 1e9}
+    pk, kind = peaks()
+    for v in res.values():
+        v["frac_of_hbm"] = v["GB/s"] / pk["hbm_gbs"]
+    res["peak_hbm_gbs"] = pk["hbm_gbs"]
+    res["peak_source"] = kind
+    hr.close()
+    hw.close()
+    return res
 
 
 # ---------------------------------------------------------------------- oracle arm
@@ -402,6 +519,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end pass")
+    ap.add_argument("--no-hbm", action="store_true", help="skip the HBM-bound kernel measurements")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -60,24 +60,41 @@ def _mix64_np(z: np.ndarray) -> np.ndarray:
     return z ^ (z >> np.uint64(31))
 
 
+def _bits_of(k: np.uint64, n: np.ndarray) -> np.ndarray:
+    """bf16 bits of the elements with (uint64) indices n of the stream with key k."""
+    g = np.uint64(GOLDEN)
+    s = np.zeros(n.shape, dtype=np.int64)
+    for r in range(3):
+        w = _mix64_np(k + (np.uint64(3) * n + np.uint64(r + 1)) * g)
+        for lane in range(4):
+            s += ((w >> np.uint64(16 * lane)) & np.uint64(0xFFFF)).astype(np.int64)
+    x = ((s - IRWIN_HALL_CENTRE).astype(np.float32) * np.float32(1.0 / 65536.0))
+    u = x.view(np.uint32).astype(np.uint64)
+    u = (u + np.uint64(0x7FFF) + ((u >> np.uint64(16)) & np.uint64(1))) >> np.uint64(16)
+    return u.astype(np.uint16)
+
+
 def normal_bf16_bits(key: int, start: int, count: int, block: int = 1 << 16) -> np.ndarray:
     """bf16 bit patterns (uint16) of elements ``start .. start+count-1`` of stream ``key``."""
     out = np.empty(count, dtype=np.uint16)
     k = np.uint64(key & MASK64)
-    g = np.uint64(GOLDEN)
     with np.errstate(over="ignore"):
         for b0 in range(0, count, block):
             n = np.arange(start + b0, start + min(count, b0 + block), dtype=np.uint64)
-            s = np.zeros(n.shape, dtype=np.int64)
-            for r in range(3):
-                w = _mix64_np(k + (np.uint64(3) * n + np.uint64(r + 1)) * g)
-                for lane in range(4):
-                    s += ((w >> np.uint64(16 * lane)) & np.uint64(0xFFFF)).astype(np.int64)
-            x = ((s - IRWIN_HALL_CENTRE).astype(np.float32) * np.float32(1.0 / 65536.0))
-            u = x.view(np.uint32).astype(np.uint64)
-            u = (u + np.uint64(0x7FFF) + ((u >> np.uint64(16)) & np.uint64(1))) >> np.uint64(16)
-            out[b0:b0 + len(n)] = u.astype(np.uint16)
+            out[b0:b0 + len(n)] = _bits_of(k, n)
     return out
+
+
+def normal_bf16_bits_at(key: int, index, block: int = 1 << 16) -> np.ndarray:
+    """bf16 bit patterns of the elements at the given indices (any shape) of stream ``key``."""
+    idx = np.asarray(index, dtype=np.uint64)
+    flat = idx.reshape(-1)
+    out = np.empty(flat.shape, dtype=np.uint16)
+    k = np.uint64(key & MASK64)
+    with np.errstate(over="ignore"):
+        for b0 in range(0, flat.size, block):
+            out[b0:b0 + block] = _bits_of(k, flat[b0:b0 + block])
+    return out.reshape(idx.shape)
 
 
 # ---------------------------------------------------------------- CUDA twin

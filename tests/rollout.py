@@ -181,3 +181,84 @@ class Rollout:
             if f >= 0:
                 assert s == (f if f < S else S + (f - S) % R)
         assert self.h.frames_committed(layer) == self.f0[layer]
+
+
+def host_bits_heads(cfg: Config, layer, chunk, call, tag, n_tok, heads):
+    """bits of the selected heads only, [n_tok, len(heads), 128] (element (t, h, c) of the
+    full [n_tok, H, 128] tensor sits at index (t * H + h) * 128 + c of its stream)."""
+    t = np.arange(n_tok, dtype=np.int64)[:, None, None]
+    h = np.asarray(heads, dtype=np.int64)[None, :, None]
+    c = np.arange(128, dtype=np.int64)[None, None, :]
+    return synth.normal_bf16_bits_at(key(cfg, layer, chunk, call, tag), (t * cfg.H + h) * 128 + c)
+
+
+class SampledRollout:
+    """Full-size rollout: the library runs every head, the oracle the sampled heads only
+    (heads never interact), so the oracle's cost stays in seconds at the real sizes."""
+
+    def __init__(self, cfg: Config, torch, heads, layer=0):
+        import rolling_kv_chunked_b200 as rkv
+        self.cfg, self.torch, self.heads, self.layer = cfg, torch, list(heads), layer
+        c = cfg
+        self.h = rkv.RollingKV(c.layers, c.H, 128, c.T, c.W, c.S, c.rope_mode)
+        self.h.set_rope_grid(c.grid_h, c.grid_w, 1.0e4, (22, 21, 21))
+        self.orc = OracleLayer(len(self.heads), 128, c.T, c.grid_h, c.grid_w, c.W, c.S, c.rope_mode)
+        self.f0 = 0
+        if c.refs:
+            k = dev_tensor(torch, c, layer, -1, 0, "k", c.refs * c.T)
+            v = dev_tensor(torch, c, layer, -1, 0, "v", c.refs * c.T)
+            self.h.write_chunk(layer, k, v, c.refs, 0)
+            self.orc.write_chunk(host_bits_heads(c, layer, -1, 0, "k", c.refs * c.T, self.heads),
+                                 host_bits_heads(c, layer, -1, 0, "v", c.refs * c.T, self.heads), c.refs, 0)
+            self.f0 = c.refs
+
+    def run_chunk(self, chunk, rows=None, stats=None):
+        """All calls of one chunk; with ``rows`` the first read and the commit are compared
+        on those query rows of the sampled heads."""
+        c, torch = self.cfg, self.torch
+        out = torch.empty((c.Lq, c.H, 128), dtype=torch.bfloat16, device="cuda")
+        for call in range(c.reads + 1):
+            commit = call == c.reads
+            q, k, v = (dev_tensor(torch, c, self.layer, chunk, call, t, c.Lq) for t in ("q", "k", "v"))
+            self.h.chunk_attention(self.layer, q, k, v, out, c.C, self.f0, commit)
+            if rows is not None and call in (0, c.reads):
+                qb, kb, vb = (host_bits_heads(c, self.layer, chunk, call, t, c.Lq, self.heads) for t in ("q", "k", "v"))
+                ref = self.orc.chunk_attention(qb, kb, vb, c.C, self.f0, commit, rows=rows)
+                got = to_bits(out)[np.asarray(rows)][:, self.heads]
+                r = assert_close(got, ref, f"{c.name} chunk {chunk} call {call}")
+                if stats is not None:
+                    stats.append(r)
+            elif commit:
+                self.orc.write_chunk(host_bits_heads(c, self.layer, chunk, call, "k", c.Lq, self.heads),
+                                     host_bits_heads(c, self.layer, chunk, call, "v", c.Lq, self.heads), c.C, self.f0)
+        self.f0 += c.C
+
+    def check_cache(self):
+        c, torch = self.cfg, self.torch
+        frames = self.h.slot_frames(self.layer)
+        kp, vp = self.h.cache_ptrs(self.layer)
+        n_el = c.H * c.W * c.T * 128
+        hs = torch.tensor(self.heads, device="cuda")
+        k_all = _wrap(torch, kp, n_el).view(c.H, c.W * c.T, 128).index_select(0, hs)
+        v_all = _wrap(torch, vp, n_el).view(c.H, c.W * c.T, 128).index_select(0, hs)
+        held = sorted((f, s) for s, f in enumerate(frames) if f >= 0)
+        assert [f for f, _ in held] == self.orc.logical_frames()
+        ok, ov = self.orc.logical_kv_bits()
+        kb = to_bits(torch.cat([k_all[:, s * c.T:(s + 1) * c.T].permute(1, 0, 2) for _, s in held]))
+        vb = to_bits(torch.cat([v_all[:, s * c.T:(s + 1) * c.T].permute(1, 0, 2) for _, s in held]))
+        assert np.array_equal(kb, ok) and np.array_equal(vb, ov)
+        S, R = c.S, c.W - c.S
+        for s, f in enumerate(frames):
+            if f >= 0:
+                assert s == (f if f < S else S + (f - S) % R)
+        assert self.h.frames_committed(self.layer) == self.f0
+
+
+def sample_rows(Lq, n=96, seed=0):
+    """Random query rows plus the edges of every 128-row tile and of the chunk."""
+    rng = np.random.default_rng(seed)
+    edges = {0, 1, Lq - 2, Lq - 1}
+    for b in range(128, Lq, 128):
+        edges.update({b - 1, b})
+    rows = set(rng.choice(Lq, size=min(n, Lq), replace=False).tolist()) | {e for e in edges if 0 <= e < Lq}
+    return np.array(sorted(rows))

@@ -166,3 +166,25 @@ def test_host_errors_launch_nothing():
     assert torch.count_nonzero(out).item() == 0
     assert h.frames_committed(0) == 0 and h.slot_frames(0) == [-1] * cfg.W
     h.close()
+
+
+def test_expired_wait_reports_timeout_and_context_survives():
+    """A 1 ns cap makes the kernel's first unsatisfied wait expire: the call must come back
+    (no hang, no trap) with RKV_ERR_TIMEOUT from the status word, and the next call with the
+    normal cap must be correct."""
+    cfg = Config("timeout", 11, H=2, grid_h=4, grid_w=4, C=2, W=6, S=2, rope_mode=ABS)
+    h = rkv.RollingKV(1, cfg.H, 128, cfg.T, cfg.W, cfg.S, cfg.rope_mode)
+    h.set_rope_grid(cfg.grid_h, cfg.grid_w)
+    q, k, v = (dev_tensor(torch, cfg, 0, 0, 0, t, cfg.Lq) for t in ("q", "k", "v"))
+    out = torch.zeros((cfg.Lq, cfg.H, 128), dtype=torch.bfloat16, device="cuda")
+    h.set_wait_limit(1)
+    h.chunk_attention(0, q, k, v, out, cfg.C, 0, False)
+    assert h.poll_device_status() == rkv.ERR_TIMEOUT
+    assert h.poll_device_status() == rkv.OK          # the word is cleared by the poll
+    h.set_wait_limit(2_000_000_000)
+    h.chunk_attention(0, q, k, v, out, cfg.C, 0, False)
+    assert h.poll_device_status() == rkv.OK
+    orc = OracleLayer(cfg.H, 128, cfg.T, cfg.grid_h, cfg.grid_w, cfg.W, cfg.S, cfg.rope_mode)
+    ref = orc.chunk_attention(to_bits(q), to_bits(k), to_bits(v), cfg.C, 0, False)
+    assert_close(to_bits(out), ref, "after timeout")
+    h.close()

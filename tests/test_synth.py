@@ -43,3 +43,10 @@ def test_moments():
     assert abs(x.mean()) < 0.01
     assert abs(x.var() - 1.0) < 0.02
     assert np.all(np.abs(x) <= 6.0)
+
+
+def test_indexed_form_matches_contiguous():
+    key = synth.stream_key(4, 2)
+    full = synth.normal_bf16_bits(key, 0, 30000)
+    idx = np.array([[0, 7, 29999], [12345, 3, 3]])
+    assert np.array_equal(synth.normal_bf16_bits_at(key, idx), full[idx])
