@@ -28,6 +28,11 @@ __device__ __forceinline__ uint16_t f64_to_bf16_rne(double x) {
   return static_cast<uint16_t>(u);
 }
 
+// bf16 -> fp64, exact.
+__device__ __forceinline__ double bf16_to_f64(uint32_t b) {
+  return static_cast<double>(bf16_to_f32(static_cast<uint16_t>(b)));
+}
+
 // x0 = xt - sigma * v; xt' = (1 - sigma') * x0 + sigma' * eps, in fp64 with every
 // operation rounded on its own (no fused multiply-add).
 struct FlowStep {
@@ -38,6 +43,12 @@ struct FlowStep {
     const double x0 = __dsub_rn(xt, __dmul_rn(sigma, v));
     x0_out = f64_to_bf16_rne(x0);
     if (renoise) xn_out = f64_to_bf16_rne(__dadd_rn(__dmul_rn(one_minus_next, x0), __dmul_rn(sigma_next, eps)));
+  }
+  // the same on bf16 bit patterns (low 16 bits of each argument)
+  __device__ __forceinline__ void apply_bits(uint32_t xt, uint32_t v, uint32_t eps, uint16_t& x0_out,
+                                             uint16_t& xn_out) const {
+    apply(bf16_to_f64(xt & 0xFFFFu), bf16_to_f64(v & 0xFFFFu), renoise ? bf16_to_f64(eps & 0xFFFFu) : 0.0, x0_out,
+          xn_out);
   }
 };
 

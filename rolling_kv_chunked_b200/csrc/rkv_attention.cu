@@ -426,8 +426,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int q = 0; q < 4; ++q) {
                 const uint32_t vw = ob[4 * v + q];
                 uint16_t a0, a1, b0 = 0, b1 = 0;
-                step.apply(bf16_to_f32(xw[q] & 0xFFFFu), bf16_to_f32(vw & 0xFFFFu), bf16_to_f32(ew[q] & 0xFFFFu), a0, b0);
-                step.apply(bf16_to_f32(xw[q] >> 16), bf16_to_f32(vw >> 16), bf16_to_f32(ew[q] >> 16), a1, b1);
+                step.apply_bits(xw[q], vw, ew[q], a0, b0);
+                step.apply_bits(xw[q] >> 16, vw >> 16, ew[q] >> 16, a1, b1);
                 o0[q] = static_cast<uint32_t>(a0) | (static_cast<uint32_t>(a1) << 16);
                 o1[q] = static_cast<uint32_t>(b0) | (static_cast<uint32_t>(b1) << 16);
               }

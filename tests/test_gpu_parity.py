@@ -188,3 +188,28 @@ def test_expired_wait_reports_timeout_and_context_survives():
     ref = orc.chunk_attention(to_bits(q), to_bits(k), to_bits(v), cfg.C, 0, False)
     assert_close(to_bits(out), ref, "after timeout")
     h.close()
+
+
+def test_flow_epilogue_all_finite_bit_patterns():
+    """Inputs drawn uniformly over every finite bf16 bit pattern (zeros, subnormals, the
+    largest magnitudes): x0 and xt' must equal the oracle's fp64 result rounded to nearest
+    even bit for bit, including rounding ties, subnormal results and overflow to infinity."""
+    rng = np.random.default_rng(123)
+    n = 1 << 20
+    def finite_bits():
+        b = rng.integers(0, 1 << 16, size=n, dtype=np.uint32).astype(np.uint16)
+        exp = (b.astype(np.uint32) >> 7) & 0xFF
+        b[exp == 0xFF] &= 0x807F          # map inf / nan patterns to finite ones
+        return b
+    xb, vb, eb = finite_bits(), finite_bits(), finite_bits()
+    dev = lambda b: torch.from_numpy(b.view(np.int16).copy()).cuda().view(torch.bfloat16)
+    xt, v, eps = dev(xb), dev(vb), dev(eb)
+    for s, sn in [(1.0, 0.75), (0.75, 0.5), (0.5, 0.25), (0.25, -1.0), (0.5, 0.0)]:
+        x0 = torch.empty_like(xt)
+        xn = torch.empty_like(xt)
+        rkv.flow_x0_renoise(xt, v, eps, s, sn, x0, xn if sn >= 0 else None)
+        torch.cuda.synchronize()
+        rx0, rxn = oflow.x0_renoise_bf16(xb, vb, eb, s, sn)
+        assert np.array_equal(to_bits(x0), rx0), s
+        if sn >= 0:
+            assert np.array_equal(to_bits(xn), rxn), s
