@@ -131,6 +131,25 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# ---------------------------------------------------------------------- ranks
+def reduce_max(x, device="cpu"):
+    """Max of x over all ranks (x itself without a process group): every multi-GPU time
+    reported is the slowest rank's."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_env():
+    """(world, rank, local_rank) from the torchrun environment (1, 0, 0 without it)."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
 # ---------------------------------------------------------------------- CUDA arm
 def visible_keys(cfg, committed, f0):
     import rolling_kv_chunked_b200 as rkv
@@ -145,9 +164,7 @@ def run_rkv(args):
     import rolling_kv_chunked_b200 as rkv
     import synth
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
     torch.cuda.set_device(local)
     if world > 1:
         from datetime import timedelta
@@ -250,10 +267,7 @@ def run_rkv(args):
     status = h.poll_device_status(sp)
     if status != rkv.OK:
         raise RuntimeError("device wait expired in the timed region")
-    if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = reduce_max(ms, "cuda")
     tokens = 5 * Lq * args.steps * world
     value = tokens / (ms / 1e3)
 
@@ -362,11 +376,7 @@ def run_e2e(args, torch, dist, world, pool, step, tokens):
     comp.wait_stream(d2h_s)
     e1.record(comp)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = reduce_max(e0.elapsed_time(e1), "cuda")
     return {"value": tokens / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": e2e_ms / args.steps, "overlap": "h2d / kernels / d2h on three streams, double-buffered"}
 
@@ -479,10 +489,9 @@ def cpu_baseline(cfg, budget_s=10.0, heads=2):
 
 
 def run_reference(args):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
+    world, rank, _ = rank_env()
     if rank != 0:
-        return
+        return                     # the oracle arm runs on rank 0 only; other ranks exit 0
     cfg = CONFIGS[args.config]
     orc, q, f0 = _oracle_steady_layer(cfg)
     C, H = cfg["C"], cfg["H"]
