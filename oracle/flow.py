@@ -13,6 +13,7 @@ The sigma schedule is sigma = t / 1000 for the distilled timesteps
 Operation order (no fused multiply-add; numpy does not contract):
     x0  = xt - (sigma * v)
     xt' = ((1 - sigma') * x0) + (sigma' * eps)
+    v   = u + (scale * (c - u))          (guided prediction, when CFG is used)
 x0 used for renoising is the fp64 value, not its bf16 rounding.
 """
 from __future__ import annotations
@@ -37,6 +38,25 @@ def x0_renoise_f64(xt, v, eps, sigma: float, sigma_next: float):
         return x0, None
     eps = np.asarray(eps, dtype=np.float64)
     return x0, (1.0 - sigma_next) * x0 + sigma_next * eps
+
+
+def cfg_combine_f64(v_cond, v_uncond, scale: float):
+    """Classifier-free guidance: v = v_uncond + scale * (v_cond - v_uncond), fp64, no FMA.
+
+    The causal pre-training mode runs 40 steps with CFG scale 5.0, i.e. two DiT forwards per
+    step, one per KV cache ([P2] §为什么需要: "40 步 ... scale5.0 ... 40 × 2 = 80 次";
+    [P3] §两种推理模式: cond / uncond each keep their own KV cache)."""
+    c = np.asarray(v_cond, dtype=np.float64)
+    u = np.asarray(v_uncond, dtype=np.float64)
+    return u + scale * (c - u)
+
+
+def cfg_x0_renoise_bf16(xt_bits, vc_bits, vu_bits, eps_bits, scale: float, sigma: float, sigma_next: float):
+    """Guided flow prediction, then the x0 / renoise step; bf16 in / out, fp64 arithmetic."""
+    v = cfg_combine_f64(bf16.to_f64(vc_bits), bf16.to_f64(vu_bits), scale)
+    x0, xn = x0_renoise_f64(bf16.to_f64(xt_bits), v, None if sigma_next < 0 else bf16.to_f64(eps_bits),
+                            sigma, sigma_next)
+    return bf16.from_f64(x0), (None if xn is None else bf16.from_f64(xn))
 
 
 def x0_renoise_bf16(xt_bits, v_bits, eps_bits, sigma: float, sigma_next: float):

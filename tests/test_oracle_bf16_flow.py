@@ -112,3 +112,30 @@ def test_flow_special_cases():
 
 def test_sigma_schedule():
     assert flow.sigmas() == [1.0, 0.75, 0.5, 0.25]
+
+
+def test_cfg_golden():
+    for row in _rows("cfg_combine.txt"):
+        left, right = row.split("|")
+        c, u, sc, xt, eps, s, sn = map(float, left.split())
+        v_exp, x0_exp, xn_exp = right.split()
+        assert float(flow.cfg_combine_f64(c, u, sc)) == float(v_exp)
+        enc = lambda a: bf16.from_f64(np.array([a]))
+        bx0, bxn = flow.cfg_x0_renoise_bf16(enc(xt), enc(c), enc(u), enc(eps), sc, s, sn)
+        assert bf16.to_f64(bx0)[0] == float(x0_exp)
+        if xn_exp == "none":
+            assert bxn is None
+        else:
+            assert bf16.to_f64(bxn)[0] == float(xn_exp)
+
+
+def test_cfg_special_cases():
+    rng = np.random.default_rng(5)
+    # bf16-representable inputs: c - u is exact in fp64, so scale 1 / 0 return c / u exactly
+    c = bf16.to_f64(bf16.from_f64(rng.standard_normal(5000)))
+    u = bf16.to_f64(bf16.from_f64(rng.standard_normal(5000)))
+    assert np.array_equal(flow.cfg_combine_f64(c, u, 1.0), c)
+    assert np.array_equal(flow.cfg_combine_f64(c, u, 0.0), u)
+    assert np.array_equal(flow.cfg_combine_f64(c, c, 5.0), c)      # no disagreement, no guidance
+    # linear in the scale: v(s) - u = s * (c - u)
+    assert np.allclose(flow.cfg_combine_f64(c, u, 5.0) - u, 5.0 * (c - u), rtol=0, atol=1e-14)
