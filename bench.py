@@ -12,7 +12,10 @@ to steady state (full window, evictions firing) before warm-up.
 Metric: query tokens / s per layer (5 * Lq per step), whole job over all ranks.
 Multi-GPU: independent replicas (one layer each), no data-path collective.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config abot|480p|720p] [--impl rkv|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config abot|480p|720p|abot_cfg] [--impl rkv|reference]
+
+``--config abot_cfg`` measures the guided (classifier-free guidance) mode instead: two caches,
+40 guided steps per chunk with the guidance combine fused into the unconditional read.
 """
 from __future__ import annotations
 
@@ -46,27 +49,46 @@ CONFIGS = {
                           "[14400 x 5120] latent, 4 denoise reads + 1 commit per chunk",
                  H=40, gh=45, gw=80, C=4, W=18, S=6, refs=0, mode=0),
 }
+# classifier-free guidance (causal pre-training mode): a second cache per layer for the
+# unconditional branch, 40 guided steps per chunk, guidance scale 5.0
+CFG_CONFIGS = {
+    "abot_cfg": dict(CONFIGS["abot"], workload=(
+        "ABot-style shape in the guided causal pre-training mode: 1 layer, two rolling caches (conditional, "
+        "unconditional), H=24, d=128, 880 tokens/frame (22x40 grid), chunk 3 frames (2640 queries), window 21 "
+        "frames (18480 keys), 5 sink reference frames, relative RoPE; per chunk 40 guided steps (conditional read, "
+        "then unconditional read with the guidance combine and x0 / renoise fused, scale 5.0) + 2 commits")),
+}
+CFG_SCALE = 5.0
+CFG_STEPS = 40
 SIGMAS = [1.0, 0.75, 0.5, 0.25]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-ATTN_SRC = os.path.join(ROOT, "rolling_kv_chunked_b200", "csrc", "rkv_attention.cu")
+# every source file the attention kernel is compiled from
+ATTN_SRCS = [os.path.join(ROOT, "rolling_kv_chunked_b200", "csrc", f)
+             for f in ("rkv_attention.cu", "numeric.cuh", "ptx_sm100.cuh", "rkv_internal.h")]
+
+
+def attention_source_sha256():
+    import hashlib
+    h = hashlib.sha256()
+    for path in ATTN_SRCS:
+        with open(path, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
 
 
 def profiled_traffic(config_name):
     """DRAM bytes per attention launch from the committed ncu record of this workload, if that
-    record was taken on the current kernel source (same sha256), else None."""
-    import hashlib
+    record was taken on the current kernel sources (same sha256), else None."""
     rec = os.path.join(ROOT, "profiles", f"chunk_attention_{config_name}.traffic.json")
     if not os.path.exists(rec):
         return None, None
     with open(rec) as fh:
         r = json.load(fh)
-    with open(ATTN_SRC, "rb") as fh:
-        sha = hashlib.sha256(fh.read()).hexdigest()
-    if r.get("kernel_source_sha256") != sha:
+    if r.get("kernel_sources_sha256") != attention_source_sha256():
         return None, "kernel changed since the counters were taken"
-    return r["dram_bytes_per_launch"], rec
+    return r["dram_bytes_per_launch"], os.path.relpath(rec, ROOT)
 
 
 def peaks():
@@ -310,6 +332,146 @@ def run_rkv(args):
         print(json.dumps(result), flush=True)
 
 
+def run_cfg(args):
+    """Guided mode on one GPU: one step = one chunk = 40 x (conditional read, unconditional read
+    with the fused guidance + x0 / renoise epilogue) + the commit of each branch (82 attention
+    launches). Device-timed with inputs resident in HBM."""
+    import torch
+
+    import rolling_kv_chunked_b200 as rkv
+    import synth
+
+    world, rank, local = rank_env()
+    if world > 1:
+        raise SystemExit("the guided workload is measured on one GPU")
+    torch.cuda.set_device(local)
+    cfg = CFG_CONFIGS[args.config]
+    H, C, W, S = cfg["H"], cfg["C"], cfg["W"], cfg["S"]
+    T = cfg["gh"] * cfg["gw"]
+    Lq = C * T
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+    hs = [rkv.RollingKV(1, H, 128, T, W, S, cfg["mode"]) for _ in range(2)]
+    for h in hs:
+        h.set_rope_grid(cfg["gh"], cfg["gw"])
+
+    def fill(t, *fields):
+        synth.fill_normal_bf16_cuda(t.data_ptr(), t.numel(), synth.stream_key(rank, 76, *fields), 0, sp)
+        return t
+
+    bf = dict(dtype=torch.bfloat16, device="cuda")
+    n_sets = 5      # q/k/v sets per branch, cycled over the steps (each set 49 MB at this size)
+    qkv = [[[fill(torch.empty((Lq, H, 128), **bf), b, i, t) for t in range(3)] for i in range(n_sets)]
+           for b in range(2)]
+    xt0 = fill(torch.empty((Lq, H * 128), **bf), 9, 0, 4)
+    eps = [fill(torch.empty((Lq, H * 128), **bf), 9, i, 5) for i in range(2)]
+    outs = [torch.empty((Lq, H, 128), **bf) for _ in range(2)]
+    x0 = torch.empty((Lq, H * 128), **bf)
+    xn = [torch.empty((Lq, H * 128), **bf) for _ in range(2)]
+    sig = [1.0 - k / CFG_STEPS for k in range(CFG_STEPS)] + [-1.0]
+    state = {"f0": 0}
+
+    def step():
+        f0 = state["f0"]
+        xt = xt0
+        for k in range(CFG_STEPS):
+            a, b = qkv[0][k % (n_sets - 1)], qkv[1][k % (n_sets - 1)]
+            sn = sig[k + 1]
+            nxt = xn[k % 2] if sn >= 0 else None
+            hs[0].chunk_attention(0, *a, outs[0], C, f0, False, stream=sp)
+            hs[1].chunk_attention(0, *b, outs[1], C, f0, False, stream=sp,
+                                  flow=dict(xt=xt, eps=eps[k % 2] if sn >= 0 else None, sigma=sig[k],
+                                            sigma_next=sn, x0_out=x0, xt_next_out=nxt, v_cond=outs[0],
+                                            cfg_scale=CFG_SCALE))
+            if nxt is not None:
+                xt = nxt
+        for br in range(2):
+            hs[br].chunk_attention(0, *qkv[br][n_sets - 1], outs[br], C, f0, True, stream=sp)
+        state["f0"] = f0 + C
+
+    if cfg["refs"]:
+        for br in range(2):
+            kr = fill(torch.empty((cfg["refs"] * T, H, 128), **bf), 99, br, 2)
+            vr = fill(torch.empty((cfg["refs"] * T, H, 128), **bf), 99, br, 3)
+            hs[br].write_chunk(0, kr, vr, cfg["refs"], 0, stream=sp)
+        state["f0"] = cfg["refs"]
+    for i in range(math.ceil((W - S) / C) + 1):
+        for br in range(2):
+            hs[br].chunk_attention(0, *qkv[br][n_sets - 1], outs[br], C, state["f0"], True, stream=sp)
+        state["f0"] += C
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    calls = 2 * CFG_STEPS + 2
+    flops, f = 0.0, state["f0"]
+    for _ in range(args.steps):
+        flops += calls * 4.0 * H * 128 * Lq * visible_keys(cfg, f, f)
+        f += C
+    gpu_id = None
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
+    except Exception:
+        gpu_id = None
+    clocks = ClockSampler(gpu_id)
+    torch.cuda.synchronize()
+    for h in hs:
+        h.timing_begin(calls * args.steps)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    kernel_ms = hs[0].timing_end(calls * args.steps) + hs[1].timing_end(calls * args.steps)
+    clk = clocks.stop()
+    ms = ev0.elapsed_time(ev1)
+    for h in hs:
+        if h.poll_device_status(sp) != rkv.OK:
+            raise RuntimeError("device wait expired in the timed region")
+    tokens = calls * Lq * args.steps
+    pk, pk_kind = peaks()
+    achieved = flops / (sum(kernel_ms) / 1e3) / 1e12 if kernel_ms else None
+    peak = pk["bf16_tflops_sustained"]
+
+    # the standalone guided epilogue (K4 with guidance): 4 bf16 reads + 2 bf16 writes per element
+    n = Lq * H * 128
+    n_ep = max(2, -(-int(320e6) // (n * 2 * 6)))
+    ep_sets = [[fill(torch.empty(n, **bf), 50 + i, j) for j in range(6)] for i in range(n_ep)]
+    s_ = lambda i: ep_sets[i % n_ep]
+    rkv.flow_cfg_x0_renoise(*s_(0)[:4], CFG_SCALE, 1.0, 0.975, s_(0)[4], s_(0)[5], stream=sp)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(20):
+        rkv.flow_cfg_x0_renoise(*s_(i)[:4], CFG_SCALE, 1.0, 0.975, s_(i)[4], s_(i)[5], stream=sp)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ep_gbs = 12 * n / (e0.elapsed_time(e1) / 20 / 1e3) / 1e9
+    result = {
+        "metric": METRIC, "value": tokens / (ms / 1e3), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": cfg["workload"], "queries_per_call": Lq, "keys_per_call": W * T,
+                   "calls_per_step": calls, "parallelism": "single GPU",
+                   "l2": "inputs larger than L2 (window K/V 227 MB per branch)"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": (achieved / peak) if achieved else None, "traffic": None,
+                     "kernel": "chunk_attention_kernel", "peak_source": f"{pk_kind} bf16_tflops_sustained",
+                     "frac_of_burst": (achieved / pk["bf16_tflops"]) if achieved else None,
+                     "mean_kernel_ms": sum(kernel_ms) / max(1, len(kernel_ms)), "launches_timed": len(kernel_ms),
+                     "flops_per_launch": flops / max(1, calls * args.steps)},
+        "e2e": None,
+        "hbm_kernels": {"flow_cfg_x0_renoise": {"bytes_per_launch": 12 * n, "GB/s": ep_gbs,
+                                                "frac_of_hbm": ep_gbs / pk["hbm_gbs"]},
+                        "peak_hbm_gbs": pk["hbm_gbs"], "peak_source": pk_kind},
+        "gpu_launches": (2 * CFG_STEPS * 2 + 2 * 2) * args.steps,
+        "clocks": clk,
+    }
+    for h in hs:
+        h.close()
+    print(json.dumps(result), flush=True)
+
+
 def run_e2e(args, torch, dist, world, pool, step, tokens):
     """The same steps through the public API with every input in pinned host memory: each
     step copies its inputs host -> device and its results (the five attention outputs and
@@ -492,7 +654,7 @@ def run_reference(args):
     world, rank, _ = rank_env()
     if rank != 0:
         return                     # the oracle arm runs on rank 0 only; other ranks exit 0
-    cfg = CONFIGS[args.config]
+    cfg = {**CONFIGS, **CFG_CONFIGS}[args.config]
     orc, q, f0 = _oracle_steady_layer(cfg)
     C, H = cfg["C"], cfg["H"]
     T = cfg["gh"] * cfg["gw"]
@@ -523,7 +685,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", default="abot", choices=sorted(CONFIGS))
+    ap.add_argument("--config", default="abot", choices=sorted(CONFIGS) + sorted(CFG_CONFIGS))
     ap.add_argument("--impl", default="rkv", choices=["rkv", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -534,6 +696,8 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.config in CFG_CONFIGS:
+        run_cfg(args)
     else:
         run_rkv(args)
 

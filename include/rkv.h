@@ -125,6 +125,26 @@ int rkv_chunk_attention_flow(rkv_handle h, int layer, const void* q, const void*
                              int commit, const rkv_flow_epilogue* epi, void* stream);
 
 /*
+ * rkv_chunk_attention_cfg_flow - the unconditional branch of a classifier-free
+ *  guidance step with the guided epilogue fused into its output store. The
+ *  causal pre-training mode samples every chunk in 40 steps with guidance
+ *  scale 5.0, two forwards per step ([P2] §为什么需要, mode table), and keeps
+ *  one KV cache per branch ([P3] §两种推理模式): create one handle per branch,
+ *  run the conditional branch with rkv_chunk_attention on its handle first,
+ *  then this call on the unconditional handle `h` with v_cond = that output.
+ *  The epilogue takes u = this call's bf16 output (the value written to
+ *  `out`), v = u + cfg_scale * (c - u) in fp64 with c = v_cond, and then
+ *  applies the step of rkv_flow_x0_renoise to v.
+ *  v_cond: [n_frames*T, H*d] bf16, device, 16-byte aligned, caller-owned, read
+ *  only; it must not overlap out. epi must be non-NULL. Other arguments and
+ *  errors as rkv_chunk_attention_flow.
+ */
+int rkv_chunk_attention_cfg_flow(rkv_handle h, int layer, const void* q, const void* k,
+                                 const void* v, void* out, int n_frames, int start_frame,
+                                 int commit, const rkv_flow_epilogue* epi, const void* v_cond,
+                                 double cfg_scale, void* stream);
+
+/*
  * rkv_rope_apply - rotate x [n_frames*T, H, d] in place with the handle's 3D
  *  RoPE. Absolute mode: t = frame index ([P3] §改造③ rope_apply(..., start_frame)).
  *  Relative mode: t = clamp(f - (window_end_frame - window_frames), 0, W-1),
@@ -146,6 +166,20 @@ int rkv_rope_apply(rkv_handle h, void* x, int n_frames, int start_frame,
 int rkv_flow_x0_renoise(const void* xt, const void* v, const void* eps, double sigma,
                         double sigma_next, void* x0_out, void* xt_next_out, long long n,
                         void* stream);
+
+/*
+ * rkv_flow_cfg_x0_renoise - classifier-free guidance combine, then the step of
+ *  rkv_flow_x0_renoise: v = v_uncond + cfg_scale * (v_cond - v_uncond) in fp64
+ *  (each operation rounded on its own), x0 = xt - sigma * v, and if
+ *  sigma_next >= 0 xt_next = (1 - sigma_next) * x0 + sigma_next * eps
+ *  ([P2] §为什么需要: causal pre-training samples with guidance scale 5.0;
+ *  [P3] §两种推理模式: a conditional and an unconditional branch). n elements,
+ *  bf16 in/out, all device pointers 16-byte aligned; eps / xt_next_out may be
+ *  NULL when sigma_next < 0. Errors: RKV_ERR_ARG, RKV_ERR_CUDA.
+ */
+int rkv_flow_cfg_x0_renoise(const void* xt, const void* v_cond, const void* v_uncond,
+                            const void* eps, double cfg_scale, double sigma, double sigma_next,
+                            void* x0_out, void* xt_next_out, long long n, void* stream);
 
 /* rkv_slot_frames - host copy of the slot -> frame map of `layer`: frames_out[W],
  *  -1 = empty. Slots [0, S) hold the sinks; frame f >= S lives in slot

@@ -50,8 +50,11 @@ _SIGS = {
     "rkv_chunk_attention": ([_vp, _c_int, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _vp], _c_int),
     "rkv_chunk_attention_flow": ([_vp, _c_int, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int,
                                   ctypes.POINTER(FlowEpilogue), _vp], _c_int),
+    "rkv_chunk_attention_cfg_flow": ([_vp, _c_int, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int,
+                                      ctypes.POINTER(FlowEpilogue), _vp, _c_dbl, _vp], _c_int),
     "rkv_rope_apply": ([_vp, _vp, _c_int, _c_int, _c_int, _vp], _c_int),
     "rkv_flow_x0_renoise": ([_vp, _vp, _vp, _c_dbl, _c_dbl, _vp, _vp, _c_ll, _vp], _c_int),
+    "rkv_flow_cfg_x0_renoise": ([_vp, _vp, _vp, _vp, _c_dbl, _c_dbl, _c_dbl, _vp, _vp, _c_ll, _vp], _c_int),
     "rkv_slot_frames": ([_vp, _c_int, _int_p], _c_int),
     "rkv_frames_committed": ([_vp, _c_int, _int_p], _c_int),
     "rkv_cache_ptrs": ([_vp, _c_int, ctypes.POINTER(_vp), ctypes.POINTER(_vp)], _c_int),
@@ -125,6 +128,14 @@ def flow_x0_renoise(xt, v, eps, sigma: float, sigma_next: float, x0_out, xt_next
            "rkv_flow_x0_renoise")
 
 
+def flow_cfg_x0_renoise(xt, v_cond, v_uncond, eps, cfg_scale: float, sigma: float, sigma_next: float, x0_out,
+                        xt_next_out=None, stream=None) -> None:
+    """v = v_uncond + cfg_scale (v_cond - v_uncond), then the x0 / renoise step of flow_x0_renoise."""
+    _check(_lib.rkv_flow_cfg_x0_renoise(_ptr(xt), _ptr(v_cond), _ptr(v_uncond), _ptr(eps), float(cfg_scale),
+                                        float(sigma), float(sigma_next), _ptr(x0_out), _ptr(xt_next_out),
+                                        xt.numel(), _stream(stream)), "rkv_flow_cfg_x0_renoise")
+
+
 class RollingKV:
     """One rkv handle: per-layer rolling caches plus the RoPE configuration."""
 
@@ -152,7 +163,9 @@ class RollingKV:
     def chunk_attention(self, layer: int, q, k, v, out, n_frames: int, start_frame: int, commit: bool,
                         stream=None, flow: dict | None = None) -> None:
         """out = attention of the chunk's queries; ``flow`` = dict(xt, eps, sigma, sigma_next, x0_out,
-        xt_next_out) fuses the x0/renoise epilogue into the output store."""
+        xt_next_out) fuses the x0/renoise epilogue into the output store. With ``v_cond`` and
+        ``cfg_scale`` in ``flow`` this call is the unconditional branch of a guided step: the epilogue
+        uses v = out + cfg_scale (v_cond - out)."""
         if flow is None:
             rc = _lib.rkv_chunk_attention(self._h, layer, _ptr(q), _ptr(k), _ptr(v), _ptr(out), n_frames,
                                           start_frame, int(bool(commit)), _stream(stream))
@@ -160,6 +173,12 @@ class RollingKV:
             return
         epi = FlowEpilogue(_ptr(flow["xt"]), _ptr(flow.get("eps")), float(flow["sigma"]),
                            float(flow["sigma_next"]), _ptr(flow["x0_out"]), _ptr(flow.get("xt_next_out")))
+        if flow.get("v_cond") is not None:
+            rc = _lib.rkv_chunk_attention_cfg_flow(self._h, layer, _ptr(q), _ptr(k), _ptr(v), _ptr(out), n_frames,
+                                                   start_frame, int(bool(commit)), ctypes.byref(epi),
+                                                   _ptr(flow["v_cond"]), float(flow["cfg_scale"]), _stream(stream))
+            _check(rc, "rkv_chunk_attention_cfg_flow")
+            return
         rc = _lib.rkv_chunk_attention_flow(self._h, layer, _ptr(q), _ptr(k), _ptr(v), _ptr(out), n_frames,
                                            start_frame, int(bool(commit)), ctypes.byref(epi), _stream(stream))
         _check(rc, "rkv_chunk_attention_flow")

@@ -50,6 +50,14 @@ struct FlowStep {
     apply(bf16_to_f64(xt & 0xFFFFu), bf16_to_f64(v & 0xFFFFu), renoise ? bf16_to_f64(eps & 0xFFFFu) : 0.0, x0_out,
           xn_out);
   }
+  // classifier-free guidance first: v = u + scale * (c - u), each operation rounded on its own,
+  // v kept in fp64 for the step
+  __device__ __forceinline__ void apply_cfg_bits(uint32_t xt, uint32_t c, uint32_t u, uint32_t eps, double scale,
+                                                 uint16_t& x0_out, uint16_t& xn_out) const {
+    const double ud = bf16_to_f64(u & 0xFFFFu);
+    const double v = __dadd_rn(ud, __dmul_rn(scale, __dsub_rn(bf16_to_f64(c & 0xFFFFu), ud)));
+    apply(bf16_to_f64(xt & 0xFFFFu), v, renoise ? bf16_to_f64(eps & 0xFFFFu) : 0.0, x0_out, xn_out);
+  }
 };
 
 }  // namespace rkv

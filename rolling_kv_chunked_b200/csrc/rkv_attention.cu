@@ -414,20 +414,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint4* ep = reinterpret_cast<const uint4*>(p.eps + base + 32 * c);
             uint4* x0p = reinterpret_cast<uint4*>(p.x0 + base + 32 * c);
             uint4* xnp = reinterpret_cast<uint4*>(p.xt_next + base + 32 * c);
+            const uint4* cp = reinterpret_cast<const uint4*>(p.v_cond + base + 32 * c);
+            const bool cfg = p.v_cond != nullptr;
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
               const uint4 xv = __ldg(xtp + v);
-              uint4 ev = make_uint4(0, 0, 0, 0);
+              uint4 ev = make_uint4(0, 0, 0, 0), cv = make_uint4(0, 0, 0, 0);
               if (step.renoise) ev = __ldg(ep + v);
+              if (cfg) cv = __ldg(cp + v);
               const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
               const uint32_t ew[4] = {ev.x, ev.y, ev.z, ev.w};
+              const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
               uint32_t o0[4], o1[4];
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
                 const uint32_t vw = ob[4 * v + q];
                 uint16_t a0, a1, b0 = 0, b1 = 0;
-                step.apply_bits(xw[q], vw, ew[q], a0, b0);
-                step.apply_bits(xw[q] >> 16, vw >> 16, ew[q] >> 16, a1, b1);
+                if (cfg) {
+                  // this launch is the unconditional branch: its output is u
+                  step.apply_cfg_bits(xw[q], cw[q], vw, ew[q], p.cfg_scale, a0, b0);
+                  step.apply_cfg_bits(xw[q] >> 16, cw[q] >> 16, vw >> 16, ew[q] >> 16, p.cfg_scale, a1, b1);
+                } else {
+                  step.apply_bits(xw[q], vw, ew[q], a0, b0);
+                  step.apply_bits(xw[q] >> 16, vw >> 16, ew[q] >> 16, a1, b1);
+                }
                 o0[q] = static_cast<uint32_t>(a0) | (static_cast<uint32_t>(a1) << 16);
                 o1[q] = static_cast<uint32_t>(b0) | (static_cast<uint32_t>(b1) << 16);
               }

@@ -404,15 +404,24 @@ RKV_API int rkv_write_chunk(rkv_handle h, int layer, const void* k, const void* 
   return RKV_OK;
 }
 
-RKV_API int rkv_chunk_attention_flow(rkv_handle h, int layer, const void* q, const void* k, const void* v, void* out,
-                                     int n_frames, int start_frame, int commit, const rkv_flow_epilogue* epi,
-                                     void* stream) {
+namespace {
+
+int chunk_attention_impl(rkv_handle h, int layer, const void* q, const void* k, const void* v, void* out,
+                         int n_frames, int start_frame, int commit, const rkv_flow_epilogue* epi,
+                         const void* v_cond, double cfg_scale, void* stream) {
   int rc = check_layer(h, layer);
   if (rc) return rc;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || n_frames <= 0) return RKV_ERR_ARG;
   if (epi != nullptr) {
     if (!aligned16(epi->xt) || !aligned16(epi->x0_out)) return RKV_ERR_ARG;
     if (epi->sigma_next >= 0.0 && (!aligned16(epi->eps) || !aligned16(epi->xt_next_out))) return RKV_ERR_ARG;
+  }
+  if (v_cond != nullptr) {
+    if (epi == nullptr || !aligned16(v_cond) || !std::isfinite(cfg_scale)) return RKV_ERR_ARG;
+    const long long bytes = static_cast<long long>(n_frames) * h->T * h->H * kHeadDim * 2;
+    const char* c0 = static_cast<const char*>(v_cond);
+    const char* o0 = static_cast<const char*>(out);
+    if (c0 < o0 + bytes && o0 < c0 + bytes) return RKV_ERR_ARG;  // v_cond must not overlap out
   }
   Layer& L = h->L[layer];
   Seg segs[rkv::kMaxSegs];
@@ -504,6 +513,8 @@ RKV_API int rkv_chunk_attention_flow(rkv_handle h, int layer, const void* q, con
     ap.xt_next = static_cast<uint16_t*>(epi->xt_next_out);
     ap.sigma = epi->sigma;
     ap.sigma_next = epi->sigma_next;
+    ap.v_cond = static_cast<const uint16_t*>(v_cond);
+    ap.cfg_scale = cfg_scale;
   } else {
     ap.sigma_next = -1.0;
   }
@@ -532,9 +543,25 @@ RKV_API int rkv_chunk_attention_flow(rkv_handle h, int layer, const void* q, con
   return RKV_OK;
 }
 
+}  // namespace
+
+RKV_API int rkv_chunk_attention_flow(rkv_handle h, int layer, const void* q, const void* k, const void* v, void* out,
+                                     int n_frames, int start_frame, int commit, const rkv_flow_epilogue* epi,
+                                     void* stream) {
+  return chunk_attention_impl(h, layer, q, k, v, out, n_frames, start_frame, commit, epi, nullptr, 0.0, stream);
+}
+
+RKV_API int rkv_chunk_attention_cfg_flow(rkv_handle h, int layer, const void* q, const void* k, const void* v,
+                                         void* out, int n_frames, int start_frame, int commit,
+                                         const rkv_flow_epilogue* epi, const void* v_cond, double cfg_scale,
+                                         void* stream) {
+  if (epi == nullptr || v_cond == nullptr) return RKV_ERR_ARG;
+  return chunk_attention_impl(h, layer, q, k, v, out, n_frames, start_frame, commit, epi, v_cond, cfg_scale, stream);
+}
+
 RKV_API int rkv_chunk_attention(rkv_handle h, int layer, const void* q, const void* k, const void* v, void* out,
                                 int n_frames, int start_frame, int commit, void* stream) {
-  return rkv_chunk_attention_flow(h, layer, q, k, v, out, n_frames, start_frame, commit, nullptr, stream);
+  return chunk_attention_impl(h, layer, q, k, v, out, n_frames, start_frame, commit, nullptr, nullptr, 0.0, stream);
 }
 
 RKV_API int rkv_rope_apply(rkv_handle h, void* x, int n_frames, int start_frame, int window_end_frame,
@@ -569,8 +596,32 @@ RKV_API int rkv_flow_x0_renoise(const void* xt, const void* v, const void* eps, 
   if (!aligned16(xt) || !aligned16(v) || !aligned16(x0_out)) return RKV_ERR_ARG;
   if (sigma_next >= 0.0 && (!aligned16(eps) || !aligned16(xt_next_out))) return RKV_ERR_ARG;
   rkv::FlowParams p;
+  std::memset(&p, 0, sizeof(p));
   p.xt = static_cast<const uint16_t*>(xt);
   p.v = static_cast<const uint16_t*>(v);
+  p.eps = static_cast<const uint16_t*>(eps);
+  p.x0 = static_cast<uint16_t*>(x0_out);
+  p.xt_next = static_cast<uint16_t*>(xt_next_out);
+  p.sigma = sigma;
+  p.sigma_next = sigma_next;
+  p.n = n;
+  return cuda_rc(rkv::launch_flow(p, static_cast<cudaStream_t>(stream)));
+}
+
+RKV_API int rkv_flow_cfg_x0_renoise(const void* xt, const void* v_cond, const void* v_uncond, const void* eps,
+                                    double cfg_scale, double sigma, double sigma_next, void* x0_out,
+                                    void* xt_next_out, long long n, void* stream) {
+  if (n < 0) return RKV_ERR_ARG;
+  if (n == 0) return RKV_OK;
+  if (!aligned16(xt) || !aligned16(v_cond) || !aligned16(v_uncond) || !aligned16(x0_out)) return RKV_ERR_ARG;
+  if (!std::isfinite(cfg_scale)) return RKV_ERR_ARG;
+  if (sigma_next >= 0.0 && (!aligned16(eps) || !aligned16(xt_next_out))) return RKV_ERR_ARG;
+  rkv::FlowParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.xt = static_cast<const uint16_t*>(xt);
+  p.v = static_cast<const uint16_t*>(v_cond);
+  p.v_uncond = static_cast<const uint16_t*>(v_uncond);
+  p.cfg_scale = cfg_scale;
   p.eps = static_cast<const uint16_t*>(eps);
   p.x0 = static_cast<uint16_t*>(x0_out);
   p.xt_next = static_cast<uint16_t*>(xt_next_out);

@@ -52,7 +52,9 @@ cudaError_t launch_frame_runs(const FrameRunParams& p, int max_tok, cudaStream_t
 // ---------------------------------------------------------------- flow epilogue
 struct FlowParams {
   const uint16_t* xt;
-  const uint16_t* v;
+  const uint16_t* v;         // the flow prediction; with guidance the conditional one
+  const uint16_t* v_uncond;  // non-null: v = v_uncond + cfg_scale * (v - v_uncond)
+  double cfg_scale;
   const uint16_t* eps;
   uint16_t* x0;
   uint16_t* xt_next;
@@ -87,6 +89,10 @@ struct AttnParams {
   uint16_t* x0;
   uint16_t* xt_next;
   double sigma, sigma_next;
+  // classifier-free guidance in the epilogue (v_cond non-null): this launch is the
+  // unconditional branch u, v = u + cfg_scale * (v_cond - u)
+  const uint16_t* v_cond;
+  double cfg_scale;
   unsigned* status;
   unsigned long long wait_limit_ns;
 };

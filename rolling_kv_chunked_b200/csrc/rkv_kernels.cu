@@ -1,7 +1,8 @@
 // Memory-bound kernels of the rolling-cache path:
 //  * frame runs: the commit / write-back copy into the ring (K1) and the 3D RoPE
 //    rotation of queries, chunk keys and (relative mode) the visible window (K3);
-//  * the fp64 flow-matching x0 / renoise epilogue (K4).
+//  * the fp64 flow-matching x0 / renoise epilogue (K4), optionally preceded by the
+//    classifier-free guidance combine of a conditional and an unconditional prediction.
 // All move 16-byte vectors (8 bf16) per thread with grid-stride loops sized to
 // the SM count. Measured on B200 at the 720p sizes: commit copy 92 %, RoPE 84 %,
 // epilogue about 70 % of the measured HBM copy bandwidth.
@@ -98,16 +99,25 @@ __global__ void __launch_bounds__(256) frame_runs_kernel(const __grid_constant__
   }
 }
 
-__device__ __forceinline__ uint4 flow_x0(const FlowStep& step, uint4 xt, uint4 v, uint4 e, uint4& xn) {
+// kCfg: v is the conditional prediction and u the unconditional one
+template <bool kCfg>
+__device__ __forceinline__ uint4 flow_x0(const FlowStep& step, double scale, uint4 xt, uint4 v, uint4 u, uint4 e,
+                                         uint4& xn) {
   const uint32_t xw[4] = {xt.x, xt.y, xt.z, xt.w};
   const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+  const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
   const uint32_t ew[4] = {e.x, e.y, e.z, e.w};
   uint32_t ow[4], nw[4];
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     uint16_t o0, o1, n0 = 0, n1 = 0;
-    step.apply_bits(xw[q], vw[q], ew[q], o0, n0);
-    step.apply_bits(xw[q] >> 16, vw[q] >> 16, ew[q] >> 16, o1, n1);
+    if (kCfg) {
+      step.apply_cfg_bits(xw[q], vw[q], uw[q], ew[q], scale, o0, n0);
+      step.apply_cfg_bits(xw[q] >> 16, vw[q] >> 16, uw[q] >> 16, ew[q] >> 16, scale, o1, n1);
+    } else {
+      step.apply_bits(xw[q], vw[q], ew[q], o0, n0);
+      step.apply_bits(xw[q] >> 16, vw[q] >> 16, ew[q] >> 16, o1, n1);
+    }
     ow[q] = static_cast<uint32_t>(o0) | (static_cast<uint32_t>(o1) << 16);
     nw[q] = static_cast<uint32_t>(n0) | (static_cast<uint32_t>(n1) << 16);
   }
@@ -116,6 +126,7 @@ __device__ __forceinline__ uint4 flow_x0(const FlowStep& step, uint4 xt, uint4 v
 }
 
 // Two 16-byte vectors per thread per iteration, all loads issued before the arithmetic.
+template <bool kCfg>
 __global__ void __launch_bounds__(256) flow_kernel(const FlowParams p) {
   FlowStep step;
   step.sigma = p.sigma;
@@ -127,6 +138,7 @@ __global__ void __launch_bounds__(256) flow_kernel(const FlowParams p) {
   const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const uint4* xtp = reinterpret_cast<const uint4*>(p.xt);
   const uint4* vp = reinterpret_cast<const uint4*>(p.v);
+  const uint4* up = reinterpret_cast<const uint4*>(p.v_uncond);
   const uint4* ep = reinterpret_cast<const uint4*>(p.eps);
   uint4* x0p = reinterpret_cast<uint4*>(p.x0);
   uint4* xnp = reinterpret_cast<uint4*>(p.xt_next);
@@ -135,18 +147,20 @@ __global__ void __launch_bounds__(256) flow_kernel(const FlowParams p) {
     const bool two = i2 < n_vec;
     const uint4 zero = make_uint4(0, 0, 0, 0);
     const uint4 xa = __ldg(xtp + i), va = __ldg(vp + i);
+    const uint4 ua = kCfg ? __ldg(up + i) : zero;
     const uint4 ea = step.renoise ? __ldg(ep + i) : zero;
-    uint4 xb = zero, vb = zero, eb = zero;
+    uint4 xb = zero, vb = zero, ub = zero, eb = zero;
     if (two) {
       xb = __ldg(xtp + i2);
       vb = __ldg(vp + i2);
+      if (kCfg) ub = __ldg(up + i2);
       if (step.renoise) eb = __ldg(ep + i2);
     }
     uint4 na, nb;
-    x0p[i] = flow_x0(step, xa, va, ea, na);
+    x0p[i] = flow_x0<kCfg>(step, p.cfg_scale, xa, va, ua, ea, na);
     if (step.renoise) xnp[i] = na;
     if (two) {
-      x0p[i2] = flow_x0(step, xb, vb, eb, nb);
+      x0p[i2] = flow_x0<kCfg>(step, p.cfg_scale, xb, vb, ub, eb, nb);
       if (step.renoise) xnp[i2] = nb;
     }
   }
@@ -155,7 +169,12 @@ __global__ void __launch_bounds__(256) flow_kernel(const FlowParams p) {
   if (gid < p.n - tail0) {
     const long long j = tail0 + gid;
     uint16_t o, nx = 0;
-    step.apply_bits(p.xt[j], p.v[j], step.renoise ? p.eps[j] : 0u, o, nx);
+    const uint32_t e = step.renoise ? p.eps[j] : 0u;
+    if (kCfg) {
+      step.apply_cfg_bits(p.xt[j], p.v[j], p.v_uncond[j], e, p.cfg_scale, o, nx);
+    } else {
+      step.apply_bits(p.xt[j], p.v[j], e, o, nx);
+    }
     p.x0[j] = o;
     if (step.renoise) p.xt_next[j] = nx;
   }
@@ -179,7 +198,11 @@ cudaError_t launch_flow(const FlowParams& p, cudaStream_t stream) {
   long long blocks = (vecs + 255) / 256;
   const long long cap = static_cast<long long>(sm_count()) * 8;
   blocks = std::max(1LL, std::min(blocks, cap));
-  flow_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
+  if (p.v_uncond != nullptr) {
+    flow_kernel<true><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
+  } else {
+    flow_kernel<false><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
+  }
   return cudaGetLastError();
 }
 
