@@ -13,7 +13,8 @@ What it computes, in the pages' order and notation, slow and obviously:
 * ``rope``      3D RoPE (t, h, w axes), absolute or relative (re-based, clamped) time ids.
 * ``attention`` softmax(Q K^T / sqrt(d)) V over the visible window, per head, fp64.
 * ``flow``      flow-matching x0 = xt - sigma * v and the renoise to the next sigma, fp64.
-* ``layer``     one layer's state machine tying the four together (reads vs commits).
+* ``layer``     one layer's state machine tying the four together (reads vs commits), and
+                the cross-attention over the cached text K/V (no positions, no mask).
 
 Pages cited (by title and section):
 

@@ -25,6 +25,10 @@ from .attention import attend
 from .cache import RollingCache
 
 
+class StateError(RuntimeError):
+    """A call that needs state not set yet (cross-attention before the text K/V)."""
+
+
 class OrderError(ValueError):
     """start_frame is not the number of frames committed so far."""
 
@@ -107,6 +111,28 @@ class OracleLayer:
             self.cache.slots = window
             self.committed += n_frames
         return out
+
+    # ------------------------------------------------------------ cross-attention
+    def set_text_kv(self, k_bits, v_bits):
+        """The text context's K and V, [n_text, H, d] bf16 bits, computed once per prompt and
+        kept for every later chunk ([P1] §核心答案 CrossAttention_KVCache; [P2] §3 cross-attn
+        cache; [P4] §一次流式生成的完整链路 step 1, 512 text tokens). The self-attention
+        cache is not touched."""
+        k = np.asarray(k_bits, dtype=np.uint16)
+        v = np.asarray(v_bits, dtype=np.uint16)
+        assert k.shape == v.shape and k.ndim == 3 and k.shape[1:] == (self.H, self.d) and k.shape[0] > 0
+        self.text_k, self.text_v = k.copy(), v.copy()
+
+    def cross_attention(self, q_bits, rows=None, heads=None):
+        """softmax(q K_text^T / sqrt(d)) V_text per head over all text tokens: no mask, no
+        positions (so no RoPE); fp64 result [len(rows), len(heads), d]."""
+        if getattr(self, "text_k", None) is None:
+            raise StateError("no text K/V set")
+        hs = list(range(self.H)) if heads is None else list(heads)
+        q = np.asarray(q_bits, dtype=np.uint16).reshape(-1, self.H, self.d)[:, hs, :]
+        if rows is not None:
+            q = q[np.asarray(rows)]
+        return attend(bf16.to_f64(q), bf16.to_f64(self.text_k[:, hs, :]), bf16.to_f64(self.text_v[:, hs, :]))
 
     def rope_apply(self, x_bits, n_frames, start_frame, window_end_frame=None):
         """RoPE of x [n_frames*T, H, d] as the standalone rotation call defines it: fp64 result.
