@@ -298,6 +298,7 @@ def run_rkv(args):
     if not args.no_e2e:
         e2e = run_e2e(args, torch, dist, world, pool, step, tokens)
     hbm = None if args.no_hbm else measure_hbm_kernels(torch, rkv, synth, cfg, rank)
+    cross = None if args.no_hbm else measure_cross_attention(torch, rkv, synth, cfg, rank)
 
     pk, pk_kind = peaks()
     traffic, traffic_src = profiled_traffic(args.config)
@@ -320,6 +321,7 @@ def run_rkv(args):
                      "flops_per_launch": flops / max(1, 5 * args.steps)},
         "e2e": e2e,
         "hbm_kernels": hbm,
+        "cross_attention": cross,
         "gpu_launches": 11 * args.steps,
         "clocks": clk,
     }
@@ -606,6 +608,46 @@ def measure_hbm_kernels(torch, rkv, synth, cfg, rank, reps=20):
     return res
 
 
+def measure_cross_attention(torch, rkv, synth, cfg, rank, n_text=512, reps=20):
+    """The cross-attention over the cached text K/V at the workload's chunk size: the chunk's
+    queries against n_text text tokens. Query / output sets are cycled so that the launches
+    together touch more than the 126 MB L2."""
+    H, C = cfg["H"], cfg["C"]
+    T = cfg["gh"] * cfg["gw"]
+    Lq = C * T
+    st = torch.cuda.current_stream()
+    sp = st.cuda_stream
+    bf = dict(dtype=torch.bfloat16, device="cuda")
+
+    def fill(t, *f):
+        synth.fill_normal_bf16_cuda(t.data_ptr(), t.numel(), synth.stream_key(rank, 89, *f), 0, sp)
+        return t
+
+    h = rkv.RollingKV(1, H, 128, T, cfg["W"], cfg["S"], cfg["mode"])
+    h.set_text_kv(0, fill(torch.empty((n_text, H, 128), **bf), 1), fill(torch.empty((n_text, H, 128), **bf), 2))
+    n_sets = max(2, -(-int(320e6) // (Lq * H * 128 * 2 * 2)))
+    qs = [fill(torch.empty((Lq, H, 128), **bf), 3, i) for i in range(n_sets)]
+    outs = [torch.empty((Lq, H, 128), **bf) for _ in range(n_sets)]
+    h.cross_attention(0, qs[0], outs[0], stream=sp)
+    torch.cuda.synchronize()
+    h.timing_begin(reps)
+    for i in range(reps):
+        h.cross_attention(0, qs[i % n_sets], outs[i % n_sets], stream=sp)
+    torch.cuda.synchronize()
+    ms = h.timing_end(reps)
+    if h.poll_device_status(sp) != rkv.OK:
+        raise RuntimeError("device wait expired in the cross-attention launches")
+    h.close()
+    sec = sum(ms) / len(ms) / 1e3
+    flops = 4.0 * H * 128 * Lq * n_text
+    bytes_ = 2 * Lq * H * 128 * 2 + 2 * n_text * H * 128 * 2
+    pk, kind = peaks()
+    return {"queries": Lq, "text_tokens": n_text, "mean_kernel_ms": sec * 1e3,
+            "TFLOP/s": flops / sec / 1e12, "frac_of_burst": flops / sec / 1e12 / pk["bf16_tflops"],
+            "GB/s": bytes_ / sec / 1e9, "frac_of_hbm": bytes_ / sec / 1e9 / pk["hbm_gbs"],
+            "flops_per_launch": flops, "bytes_per_launch": bytes_, "peak_source": kind}
+
+
 # ---------------------------------------------------------------------- oracle arm
 def _oracle_steady_layer(cfg):
     """An oracle layer holding a full steady-state window (one synthetic frame reused)."""
@@ -690,7 +732,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end pass")
-    ap.add_argument("--no-hbm", action="store_true", help="skip the HBM-bound kernel measurements")
+    ap.add_argument("--no-hbm", action="store_true",
+                    help="skip the side measurements (HBM-bound kernels, cross-attention)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

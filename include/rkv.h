@@ -42,7 +42,7 @@ extern "C" {
 #define RKV_ERR_UNSUPPORTED 4 /* d != 128, window > 256 frames, time id beyond table    */
 #define RKV_ERR_CUDA 5        /* a CUDA runtime / driver call failed                    */
 #define RKV_ERR_TIMEOUT 6     /* a bounded device wait expired (read via poll)          */
-#define RKV_ERR_STATE 7       /* call needs rkv_set_rope_grid first                     */
+#define RKV_ERR_STATE 7       /* call needs rkv_set_rope_grid (or rkv_set_text_kv) first */
 
 #define RKV_ROPE_ABSOLUTE 0   /* time id = absolute frame index                         */
 #define RKV_ROPE_RELATIVE 1   /* time id re-based to the window and clamped to [0, W-1] */
@@ -143,6 +143,36 @@ int rkv_chunk_attention_cfg_flow(rkv_handle h, int layer, const void* q, const v
                                  const void* v, void* out, int n_frames, int start_frame,
                                  int commit, const rkv_flow_epilogue* epi, const void* v_cond,
                                  double cfg_scale, void* stream);
+
+/*
+ * rkv_set_text_kv - fill the cross-attention cache of `layer` with the text
+ *  context's K and V. The text K/V are computed once per prompt and reused by
+ *  every later chunk ([P1] §核心答案 CrossAttention_KVCache; [P2] §3 cross-attn
+ *  cache; [P4] §一次流式生成的完整链路 step 1: the 512-token text embedding is
+ *  computed once, and a prompt change rebuilds only this cache while the
+ *  self-attention history stays). k_text, v_text: [n_text, H, d] bf16 device
+ *  pointers, token-major, 16-byte aligned, caller-owned, copied (bit copy) on
+ *  `stream` into library-owned [H][n_text][d] buffers, so the caller may reuse
+ *  its buffers once the copy has run on that stream. 1 <= n_text <= 65536. No
+ *  RoPE is applied (cross-attention has no positions). Growing n_text beyond
+ *  the largest value set so far on this layer reallocates and synchronises the
+ *  device. rkv_reset clears the cache. Errors: RKV_ERR_ARG, RKV_ERR_UNSUPPORTED
+ *  (n_text > 65536), RKV_ERR_CUDA.
+ */
+int rkv_set_text_kv(rkv_handle h, int layer, const void* k_text, const void* v_text, int n_text,
+                    void* stream);
+
+/*
+ * rkv_cross_attention - out = softmax(q K_text^T / sqrt(d)) V_text per head over
+ *  all n_text cached text tokens, no mask and no RoPE. q, out: [n_tokens, H, d]
+ *  bf16 device pointers, token-major, 16-byte aligned, caller-owned; any
+ *  n_tokens >= 1 (a chunk's video tokens: n_frames * T). Runs the tcgen05
+ *  attention kernel with one key segment. Needs no rope grid and no frame
+ *  order; the self-attention cache is neither read nor changed. Errors:
+ *  RKV_ERR_ARG, RKV_ERR_STATE (no text K/V set on this layer), RKV_ERR_CUDA.
+ */
+int rkv_cross_attention(rkv_handle h, int layer, const void* q, void* out, int n_tokens,
+                        void* stream);
 
 /*
  * rkv_rope_apply - rotate x [n_frames*T, H, d] in place with the handle's 3D

@@ -52,6 +52,8 @@ _SIGS = {
                                   ctypes.POINTER(FlowEpilogue), _vp], _c_int),
     "rkv_chunk_attention_cfg_flow": ([_vp, _c_int, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int,
                                       ctypes.POINTER(FlowEpilogue), _vp, _c_dbl, _vp], _c_int),
+    "rkv_set_text_kv": ([_vp, _c_int, _vp, _vp, _c_int, _vp], _c_int),
+    "rkv_cross_attention": ([_vp, _c_int, _vp, _vp, _c_int, _vp], _c_int),
     "rkv_rope_apply": ([_vp, _vp, _c_int, _c_int, _c_int, _vp], _c_int),
     "rkv_flow_x0_renoise": ([_vp, _vp, _vp, _c_dbl, _c_dbl, _vp, _vp, _c_ll, _vp], _c_int),
     "rkv_flow_cfg_x0_renoise": ([_vp, _vp, _vp, _vp, _c_dbl, _c_dbl, _c_dbl, _vp, _vp, _c_ll, _vp], _c_int),
@@ -182,6 +184,16 @@ class RollingKV:
         rc = _lib.rkv_chunk_attention_flow(self._h, layer, _ptr(q), _ptr(k), _ptr(v), _ptr(out), n_frames,
                                            start_frame, int(bool(commit)), ctypes.byref(epi), _stream(stream))
         _check(rc, "rkv_chunk_attention_flow")
+
+    def set_text_kv(self, layer: int, k_text, v_text, stream=None) -> None:
+        """Cache the text context's K and V ([n_text, H, d] each) for cross-attention."""
+        _check(_lib.rkv_set_text_kv(self._h, layer, _ptr(k_text), _ptr(v_text), k_text.shape[0], _stream(stream)),
+               "rkv_set_text_kv")
+
+    def cross_attention(self, layer: int, q, out, stream=None) -> None:
+        """out = softmax(q K_text^T / sqrt(d)) V_text over the cached text tokens; q, out [n, H, d]."""
+        _check(_lib.rkv_cross_attention(self._h, layer, _ptr(q), _ptr(out), q.shape[0], _stream(stream)),
+               "rkv_cross_attention")
 
     def rope_apply(self, x, n_frames: int, start_frame: int, window_end_frame: int = 0, stream=None) -> None:
         _check(_lib.rkv_rope_apply(self._h, _ptr(x), n_frames, start_frame, window_end_frame, _stream(stream)),

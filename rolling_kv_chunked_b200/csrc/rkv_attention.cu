@@ -11,7 +11,9 @@
 // only masking is of the ragged last tile of each segment.
 //
 // Queries and keys arrive already rotated (RoPE applied by the frame-run kernel on
-// their way into the head-major staging / rotated-K ring), V raw.
+// their way into the head-major staging / rotated-K ring), V raw. The same kernel serves
+// the cross-attention over the cached text K/V: one key segment, queries read token-major
+// straight from the caller's buffer, no rotation.
 //
 // Structure of one CTA (one head, 256 query rows = two 128-row tiles Q0, Q1):
 //   warps 0-3  softmax for Q0 (one thread per query row = TMEM lane)
@@ -219,7 +221,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_arrive_expect_tx(&bars[kBarQ], 2 * kTile);
       for (int t = 0; t < 2; ++t)
         for (int c = 0; c < 2; ++c)
-          ptx::tma_load_3d(smem + kSmemQ + t * kTile + c * kSlab, &tm_q, &bars[kBarQ], c * 64, m0 + t * kBM, head);
+          if (p.q_token_major)
+            ptx::tma_load_3d(smem + kSmemQ + t * kTile + c * kSlab, &tm_q, &bars[kBarQ], c * 64, head, m0 + t * kBM);
+          else
+            ptx::tma_load_3d(smem + kSmemQ + t * kTile + c * kSlab, &tm_q, &bars[kBarQ], c * 64, m0 + t * kBM, head);
       bool ok = true;
       int nk = 0, nv = 0;
       for (int j = 0; j < n_tiles; ++j) {

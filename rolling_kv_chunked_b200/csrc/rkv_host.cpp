@@ -52,6 +52,12 @@ struct Layer {
   long long rot_f0 = -1;       // relative mode: rotated ring valid for this (f0, C)
   int rot_c = -1;
   CUtensorMap tm_q, tm_k, tm_vc;
+  // cross-attention cache of the text context: K and V, [H][n_text][d] each
+  uint16_t* text_k = nullptr;
+  uint16_t* text_v = nullptr;
+  int n_text = 0;    // 0 = not set
+  int text_cap = 0;  // tokens the buffers can hold
+  CUtensorMap tm_tk, tm_tv;
 };
 
 }  // namespace
@@ -245,7 +251,10 @@ void free_layer(Layer& L) {
   cudaFree(L.v);
   cudaFree(L.rotk);
   cudaFree(L.qstage);
-  L.k = L.v = L.rotk = L.qstage = nullptr;
+  cudaFree(L.text_k);
+  cudaFree(L.text_v);
+  L.k = L.v = L.rotk = L.qstage = L.text_k = L.text_v = nullptr;
+  L.n_text = L.text_cap = 0;
 }
 
 int check_layer(const rkv_ctx* h, int layer) {
@@ -564,6 +573,94 @@ RKV_API int rkv_chunk_attention(rkv_handle h, int layer, const void* q, const vo
   return chunk_attention_impl(h, layer, q, k, v, out, n_frames, start_frame, commit, nullptr, nullptr, 0.0, stream);
 }
 
+RKV_API int rkv_set_text_kv(rkv_handle h, int layer, const void* k_text, const void* v_text, int n_text,
+                            void* stream) {
+  int rc = check_layer(h, layer);
+  if (rc) return rc;
+  if (!aligned16(k_text) || !aligned16(v_text) || n_text <= 0) return RKV_ERR_ARG;
+  if (n_text > rkv::kMaxTextTokens) return RKV_ERR_UNSUPPORTED;
+  Layer& L = h->L[layer];
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (n_text > L.text_cap) {
+    // earlier launches may still read the old buffers
+    if (cudaDeviceSynchronize() != cudaSuccess) return RKV_ERR_CUDA;
+    cudaFree(L.text_k);
+    cudaFree(L.text_v);
+    L.text_k = L.text_v = nullptr;
+    L.n_text = L.text_cap = 0;
+    const size_t b = static_cast<size_t>(n_text) * h->H * kHeadDim * 2;
+    if (cudaMalloc(&L.text_k, b) != cudaSuccess || cudaMalloc(&L.text_v, b) != cudaSuccess) {
+      cudaFree(L.text_k);
+      cudaFree(L.text_v);
+      L.text_k = L.text_v = nullptr;
+      return RKV_ERR_CUDA;
+    }
+    L.text_cap = n_text;
+  }
+  if (!encode_head_major(&L.tm_tk, L.text_k, n_text, h->H, rkv::kKeyBox) ||
+      !encode_head_major(&L.tm_tv, L.text_v, n_text, h->H, rkv::kKeyBox)) {
+    L.n_text = 0;
+    return RKV_ERR_CUDA;
+  }
+  // token-major [n_text, H, d] -> head-major [H][n_text][d], K and V (a bit copy)
+  FrameRunParams p = base_runs(h);
+  FrameRun r;
+  std::memset(&r, 0, sizeof(r));
+  token_major(r, true, h->H);
+  head_major(r, false, n_text);
+  r.n_tok = n_text;
+  r.src = static_cast<const uint16_t*>(k_text);
+  r.dst = L.text_k;
+  add_run(p, r);
+  r.src = static_cast<const uint16_t*>(v_text);
+  r.dst = L.text_v;
+  add_run(p, r);
+  rc = cuda_rc(rkv::launch_frame_runs(p, n_text, st));
+  if (rc) {
+    L.n_text = 0;
+    return rc;
+  }
+  L.n_text = n_text;
+  return RKV_OK;
+}
+
+RKV_API int rkv_cross_attention(rkv_handle h, int layer, const void* q, void* out, int n_tokens, void* stream) {
+  int rc = check_layer(h, layer);
+  if (rc) return rc;
+  if (!aligned16(q) || !aligned16(out) || n_tokens <= 0) return RKV_ERR_ARG;
+  if (static_cast<long long>(n_tokens) * h->H * kHeadDim >= (1LL << 40)) return RKV_ERR_UNSUPPORTED;
+  Layer& L = h->L[layer];
+  if (L.n_text <= 0) return RKV_ERR_STATE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  AttnParams ap;
+  std::memset(&ap, 0, sizeof(ap));
+  ap.q_token_major = 1;
+  ap.n_segs = 1;
+  ap.seg[0].src = 0;
+  ap.seg[0].k_row0 = 0;
+  ap.seg[0].v_row0 = 0;
+  ap.seg[0].n_rows = L.n_text;
+  ap.n_tiles = (L.n_text + rkv::kKeyBox - 1) / rkv::kKeyBox;
+  ap.H = h->H;
+  ap.Lq = n_tokens;
+  ap.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(kHeadDim)));
+  ap.out = static_cast<uint16_t*>(out);
+  ap.sigma_next = -1.0;
+  ap.status = h->status;
+  ap.wait_limit_ns = h->wait_ns;
+  CUtensorMap tm_q;
+  if (!encode_token_major(&tm_q, q, n_tokens, h->H, rkv::kQueryBox)) return RKV_ERR_CUDA;
+  const bool timed = h->timing && h->timing_n < h->timing_max;
+  if (timed && cudaEventRecord(h->ev_start[h->timing_n], st) != cudaSuccess) return RKV_ERR_CUDA;
+  rc = cuda_rc(rkv::launch_attention(tm_q, L.tm_tk, L.tm_tv, L.tm_tv, ap, st));
+  if (rc) return rc;
+  if (timed) {
+    if (cudaEventRecord(h->ev_stop[h->timing_n], st) != cudaSuccess) return RKV_ERR_CUDA;
+    ++h->timing_n;
+  }
+  return RKV_OK;
+}
+
 RKV_API int rkv_rope_apply(rkv_handle h, void* x, int n_frames, int start_frame, int window_end_frame,
                            void* stream) {
   if (h == nullptr || !aligned16(x) || n_frames <= 0 || start_frame < 0) return RKV_ERR_ARG;
@@ -669,6 +766,7 @@ RKV_API int rkv_reset(rkv_handle h) {
     std::fill(L.slot_frame.begin(), L.slot_frame.end(), -1);
     L.rot_f0 = -1;
     L.rot_c = -1;
+    L.n_text = 0;  // the text context must be set again
   }
   return cudaDeviceSynchronize() == cudaSuccess ? RKV_OK : RKV_ERR_CUDA;
 }
@@ -729,7 +827,7 @@ RKV_API const char* rkv_status_string(int status) {
     case RKV_ERR_UNSUPPORTED: return "unsupported size (d != 128, window > 256 frames or time id beyond table)";
     case RKV_ERR_CUDA: return "CUDA runtime or driver error";
     case RKV_ERR_TIMEOUT: return "a bounded device wait expired";
-    case RKV_ERR_STATE: return "rkv_set_rope_grid has not been called";
+    case RKV_ERR_STATE: return "required state not set (rkv_set_rope_grid, or rkv_set_text_kv for cross-attention)";
     default: return "unknown status";
   }
 }

@@ -14,6 +14,7 @@ constexpr int kHeadDim = 128;
 constexpr int kQueryBox = 128;
 constexpr int kKeyBox = 128;
 constexpr int kMaxRuns = 8;
+constexpr int kMaxTextTokens = 1 << 16;  // cross-attention context length limit
 constexpr int kMaxSegs = 4;
 constexpr int kTimeTable = 65536;  // time ids in [0, kTimeTable) have cos/sin rows
 
@@ -76,6 +77,7 @@ struct AttnSeg {
 };
 
 struct AttnParams {
+  int q_token_major;  // tm_q maps [Lq][H][d] (coordinates x, head, row) instead of [H][rows][d]
   AttnSeg seg[kMaxSegs];
   int n_segs;
   int n_tiles;  // sum over segments of ceil(n_rows / kKeyBox)
