@@ -56,6 +56,8 @@ constexpr int kSmemV = 4 * kTile;         // V stage 0, 1
 constexpr int kSmemBar = 6 * kTile;
 constexpr int kSmemBytes = 6 * kTile + 256 + 1024;  // tiles + barriers + alignment slack
 constexpr unsigned long long kDrainNs = 2000000000ull;
+constexpr float kLazyRescale = 8.0f;  // move the reference only when a maximum grows by more than 2^8
+constexpr float kRefSlack = 64.0f;    // largest accepted x = s * sl2 - reference in the one-pass path
 
 enum : int {
   kBarQ = 0,
@@ -143,8 +145,8 @@ __device__ __forceinline__ void exp2_poly_x2(uint64_t x2, float& y0, float& y1) 
 }
 
 // Softmax numerators of 64 keys (one half of a 128-key row): p = 2^(s * sl2 - m), rounded to
-// bf16 on the integer ALU (add half an ulp, keep the upper halves) and packed in pairs into
-// 32 TMEM columns at tP; row sums accumulate in acc.
+// bf16 (nearest even, one paired conversion) and packed in pairs into 32 TMEM columns at tP;
+// row sums (of the unrounded values) accumulate in acc.
 // kPoly: kPolyPairs of every 8 pairs take the polynomial path (full tiles only).
 #ifndef RKV_POLY_PAIRS
 #define RKV_POLY_PAIRS 1
@@ -167,9 +169,44 @@ __device__ __forceinline__ void softmax_half(const uint32_t* sh, uint64_t c2, ui
       b = ptx::ex2(x1);
     }
     acc[k & 3] = ptx::f2_add(acc[k & 3], ptx::f2_pack(a, b));
-    pk[k] = __byte_perm(__float_as_uint(a) + 0x8000u, __float_as_uint(b) + 0x8000u, 0x7632);
+    pk[k] = pack_bf16x2(a, b);
   }
   ptx::tmem_st32(tP, pk);
+}
+
+// The same numerators for a whole 64-key half computed against the running reference
+// (nm2 = -m) without storing them: packed pairs go to pk[0..31], and mx[0], mx[1] track the
+// largest x = s * sl2 - m, so that the caller can check the reference afterwards.
+template <bool kPoly>
+__device__ __forceinline__ void numerators_half(const uint32_t* sh, uint64_t c2, uint64_t nm2, uint32_t* pk,
+                                                uint64_t (&acc)[4], float (&mx)[2]) {
+#pragma unroll
+  for (int k = 0; k < kBN / 4; ++k) {
+    const uint64_t x = ptx::f2_fma(ptx::f2_pack(__uint_as_float(sh[2 * k]), __uint_as_float(sh[2 * k + 1])), c2, nm2);
+    float x0, x1, a, b;
+    ptx::f2_unpack(x, x0, x1);
+    mx[k & 1] = ptx::fmax3(mx[k & 1], x0, x1);
+    if (kPoly && (k & 7) < kPolyPairs) {
+      exp2_poly_x2(x, a, b);
+    } else {
+      a = ptx::ex2(x0);
+      b = ptx::ex2(x1);
+    }
+    acc[k & 3] = ptx::f2_add(acc[k & 3], ptx::f2_pack(a, b));
+    pk[k] = pack_bf16x2(a, b);
+  }
+}
+
+// O (this thread's row, 128 fp32 TMEM columns at tO) *= f
+__device__ __forceinline__ void scale_o(uint32_t tO, float f) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t rr[32];
+    ptx::tmem_ld32(tO + 32 * c, rr);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * f);
+    ptx::tmem_st32(tO + 32 * c, rr);
+  }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -310,8 +347,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tS = lane_base + col_s(wg);
     const uint32_t tO = lane_base + col_o(wg);
     const float sl2 = p.scale_log2;
-    float m_used = -INFINITY;
-    float l = 0.f;
+    const uint64_t c2 = ptx::f2_pack(sl2, sl2);
+    float m_used = -INFINITY;  // reference of the numerators, log2 units: p = 2^(s * sl2 - m_used)
+    float l = 0.f;             // row sum of the numerators, in the scale of the reference
+    float pend = 1.0f;         // change of reference decided on the previous tile, not yet applied
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
       ok = ptx::mbar_wait(&bars[kBarSFull + wg], j & 1, limit);
@@ -320,67 +359,103 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::tc_fence_after();
       int src, krow, vrow, valid;
       tile_of(p, j, src, krow, vrow, valid);
-      float m_tile;
-      {
-        // pass 1: the row maximum only
-        uint32_t sr[kBN];
-        ptx::tmem_ld128(tS, sr);
-        if (valid < kBN) {
+      // S(j) complete implies PV(j-1) complete: O now holds every product in the previous
+      // reference's scale, so a pending change applies to O and l together
+      if (__any_sync(0xffffffffu, pend != 1.0f)) scale_o(tO, pend);
+      l *= pend;
+      pend = 1.0f;
+      bool stored = false;
+      if (j > 0) {
+        // one pass against the running reference; the tile maximum comes out of the same
+        // pass (on the integer ALU, under the special-function-unit work) instead of a
+        // separate pass before it
+        const uint64_t nm2 = ptx::f2_pack(-m_used, -m_used);
+        uint64_t acc[4] = {0, 0, 0, 0};
+        float mx2[2] = {-INFINITY, -INFINITY};
+        uint32_t pk[kBN / 2];
 #pragma unroll
-          for (int i = 0; i < kBN; ++i)
-            if (i >= valid) sr[i] = 0xff800000u;
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t sh[kBN / 2];
+          ptx::tmem_ld64(tS + 64 * hh, sh);
+          if (valid < kBN) {
+#pragma unroll
+            for (int i = 0; i < kBN / 2; ++i)
+              if (64 * hh + i >= valid) sh[i] = 0xff800000u;
+            numerators_half<false>(sh, c2, nm2, pk + 32 * hh, acc, mx2);
+          } else {
+            numerators_half<true>(sh, c2, nm2, pk + 32 * hh, acc, mx2);
+          }
         }
-        float mq[4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint32_t* t = sr + 32 * c;
-          float m = ptx::fmax3(__uint_as_float(t[0]), __uint_as_float(t[1]), __uint_as_float(t[2]));
-#pragma unroll
-          for (int i = 3; i < 31; i += 2) m = ptx::fmax3(m, __uint_as_float(t[i]), __uint_as_float(t[i + 1]));
-          mq[c] = fmaxf(m, __uint_as_float(t[31]));
-        }
-        m_tile = ptx::fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3])) * sl2;
-      }
-      const bool need = m_tile > m_used + 8.0f;
-      float alpha = 1.0f;
-      if (need) {
-        alpha = ptx::ex2(m_used - m_tile);
-        m_used = m_tile;
-      }
-      l *= alpha;
-      if (j > 0 && __any_sync(0xffffffffu, need)) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t rr[32];
-          ptx::tmem_ld32(tO + 32 * c, rr);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
-          ptx::tmem_st32(tO + 32 * c, rr);
-        }
-      }
-      // p = 2^(s * scale_log2 - m_used), two lanes per instruction
-      const uint64_t c2 = ptx::f2_pack(sl2, sl2);
-      const uint64_t nm2 = ptx::f2_pack(-m_used, -m_used);
-      uint64_t acc[4] = {0, 0, 0, 0};
-      // pass 2: reload 64 columns at a time; P of the first half overwrites S columns
-      // 0..31, already read, the second half's loads touch columns 64..127 only
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t sh[kBN / 2];
-        ptx::tmem_ld64(tS + 64 * hh, sh);
-        if (valid < kBN) {
-#pragma unroll
-          for (int i = 0; i < kBN / 2; ++i)
-            if (64 * hh + i >= valid) sh[i] = 0xff800000u;
-          softmax_half<false>(sh, c2, nm2, tS + 32 * hh, acc);
-        } else {
-          softmax_half<true>(sh, c2, nm2, tS + 32 * hh, acc);
+        const float mx = fmaxf(mx2[0], mx2[1]);
+        // numerators up to 2^64 are exact in bf16 / fp32 range and keep O finite; a score
+        // further above the reference sends the whole warp to the exact path below, which
+        // recomputes the tile from S (not overwritten yet)
+        if (!__any_sync(0xffffffffu, mx > kRefSlack)) {
+          float rs[4];
+          ptx::f2_unpack(ptx::f2_add(acc[0], acc[1]), rs[0], rs[1]);
+          ptx::f2_unpack(ptx::f2_add(acc[2], acc[3]), rs[2], rs[3]);
+          l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+          if (mx > kLazyRescale) {  // move the reference to this tile's maximum from the next tile on
+            pend = ptx::ex2(-mx);
+            m_used += mx;
+          }
+          ptx::tmem_st64(tS, pk);
+          stored = true;
         }
       }
-      float rs[8];
-      ptx::f2_unpack(ptx::f2_add(acc[0], acc[1]), rs[0], rs[1]);
-      ptx::f2_unpack(ptx::f2_add(acc[2], acc[3]), rs[2], rs[3]);
-      l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+      if (!stored) {
+        // exact path (the first tile, or a score far above the reference): the row maximum
+        // first, then the numerators
+        float m_tile;
+        {
+          uint32_t sr[kBN];
+          ptx::tmem_ld128(tS, sr);
+          if (valid < kBN) {
+#pragma unroll
+            for (int i = 0; i < kBN; ++i)
+              if (i >= valid) sr[i] = 0xff800000u;
+          }
+          float mq[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint32_t* t = sr + 32 * c;
+            float m = ptx::fmax3(__uint_as_float(t[0]), __uint_as_float(t[1]), __uint_as_float(t[2]));
+#pragma unroll
+            for (int i = 3; i < 31; i += 2) m = ptx::fmax3(m, __uint_as_float(t[i]), __uint_as_float(t[i + 1]));
+            mq[c] = fmaxf(m, __uint_as_float(t[31]));
+          }
+          m_tile = ptx::fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3])) * sl2;
+        }
+        const bool need = m_tile > m_used + kLazyRescale;
+        float alpha = 1.0f;
+        if (need) {
+          alpha = ptx::ex2(m_used - m_tile);
+          m_used = m_tile;
+        }
+        l *= alpha;
+        if (j > 0 && __any_sync(0xffffffffu, need)) scale_o(tO, alpha);
+        const uint64_t nm2 = ptx::f2_pack(-m_used, -m_used);
+        uint64_t acc[4] = {0, 0, 0, 0};
+        // reload 64 columns at a time; P of the first half overwrites S columns 0..31,
+        // already read, the second half's loads touch columns 64..127 only
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t sh[kBN / 2];
+          ptx::tmem_ld64(tS + 64 * hh, sh);
+          if (valid < kBN) {
+#pragma unroll
+            for (int i = 0; i < kBN / 2; ++i)
+              if (64 * hh + i >= valid) sh[i] = 0xff800000u;
+            softmax_half<false>(sh, c2, nm2, tS + 32 * hh, acc);
+          } else {
+            softmax_half<true>(sh, c2, nm2, tS + 32 * hh, acc);
+          }
+        }
+        float rs[4];
+        ptx::f2_unpack(ptx::f2_add(acc[0], acc[1]), rs[0], rs[1]);
+        ptx::f2_unpack(ptx::f2_add(acc[2], acc[3]), rs[2], rs[3]);
+        l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+      }
       ptx::tmem_st_wait();
       ptx::tc_fence_before();
       ptx::mbar_arrive(&bars[kBarPFull + wg]);
