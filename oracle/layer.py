@@ -43,6 +43,7 @@ class Frame:
 class OracleLayer:
     ABSOLUTE = 0
     RELATIVE = 1
+    RELATIVE_SLOTS = 2  # relative RoPE with ids = position in the visible window (sinks 0..S-1)
 
     def __init__(self, H, d, tokens_per_frame, grid_h, grid_w, window, sink, rope_mode,
                  theta=rope.DEFAULT_THETA, pairs=rope.DEFAULT_PAIRS):
@@ -94,12 +95,18 @@ class OracleLayer:
 
         k = np.concatenate([f.k for f in window], axis=0)[:, hs, :]
         v = np.concatenate([f.v for f in window], axis=0)[:, hs, :]
-        k_ids = self.time_ids([f.frame for f in window], start_frame, n_frames)
+        if self.rope_mode == self.RELATIVE_SLOTS:
+            k_ids = rope.time_ids_slot_order(len(window))
+        else:
+            k_ids = self.time_ids([f.frame for f in window], start_frame, n_frames)
         k_pos = rope.token_positions(k_ids, self.T, self.grid_w)
         k_rot = rope.rotate(bf16.to_f64(k), k_pos, self.theta, self.pairs)
 
         q = np.asarray(q_bits, dtype=np.uint16).reshape(n_frames * self.T, self.H, self.d)[:, hs, :]
-        q_ids = self.time_ids([start_frame + i for i in range(n_frames)], start_frame, n_frames)
+        if self.rope_mode == self.RELATIVE_SLOTS:
+            q_ids = k_ids[len(window) - n_frames:]  # the chunk is the window's last n_frames frames
+        else:
+            q_ids = self.time_ids([start_frame + i for i in range(n_frames)], start_frame, n_frames)
         q_pos = rope.token_positions(q_ids, self.T, self.grid_w)
         if rows is not None:
             rows = np.asarray(rows)
@@ -138,10 +145,17 @@ class OracleLayer:
         """RoPE of x [n_frames*T, H, d] as the standalone rotation call defines it: fp64 result.
 
         Absolute mode: t = frame index. Relative mode: t = clamp(f - (window_end_frame - window),
-        0, window - 1), where window_end_frame is one past the last frame of the window."""
+        0, window - 1), where window_end_frame is one past the last frame of the window.
+        Slot-order mode: the frame's position in the window ending at window_end_frame, i.e.
+        t = f for a sink frame (f < sink) and otherwise f minus the number of non-sink frames
+        already evicted, max(0, window_end_frame - window); the result is then clamped to
+        [0, window - 1] (which only bites for frames outside that window)."""
         frames = np.arange(start_frame, start_frame + n_frames)
         if self.rope_mode == self.ABSOLUTE:
             t = rope.time_ids_absolute(frames)
+        elif self.rope_mode == self.RELATIVE_SLOTS:
+            evicted = max(0, window_end_frame - self.window)
+            t = np.clip(np.where(frames < self.sink, frames, frames - evicted), 0, self.window - 1)
         else:
             t = np.clip(frames - (window_end_frame - self.window), 0, self.window - 1)
         pos = rope.token_positions(t, self.T, self.grid_w)

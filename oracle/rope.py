@@ -19,6 +19,11 @@ start_frame=current_start_frame)``; [P4] §机制三 ``relative_rope_apply``):
 * relative: ids are re-based so that the current chunk's last frame is ``window-1`` and then
   clamped to ``[0, window-1]`` (the page's "clamp the time id to [0, 20]" for a 21-frame
   window); raw keys are cached and re-rotated with these ids on every call.
+* relative, slot order: the id is the frame's position in the visible window listed in
+  logical order (sinks, then the kept history, then the chunk): 0 .. n-1. This is the other
+  plain reading of [P4] §机制三's "query and key share one local coordinate system over the
+  current window"; it differs from the clamped re-basing only in the sink frames, which
+  keep distinct ids 0 .. S-1 instead of collapsing onto 0.
 """
 from __future__ import annotations
 
@@ -47,6 +52,11 @@ def omegas(theta=DEFAULT_THETA, pairs=DEFAULT_PAIRS) -> np.ndarray:
 
 def time_ids_absolute(frames) -> np.ndarray:
     return np.asarray(frames, dtype=np.int64)
+
+
+def time_ids_slot_order(n_visible: int) -> np.ndarray:
+    """Ids of the visible window's frames in their logical order: 0 .. n_visible-1."""
+    return np.arange(n_visible, dtype=np.int64)
 
 
 def time_ids_relative(frames, start_frame: int, n_frames: int, window: int) -> np.ndarray:
