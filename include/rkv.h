@@ -46,6 +46,9 @@ extern "C" {
 
 #define RKV_ROPE_ABSOLUTE 0   /* time id = absolute frame index                         */
 #define RKV_ROPE_RELATIVE 1   /* time id re-based to the window and clamped to [0, W-1] */
+#define RKV_ROPE_RELATIVE_SLOTS 2 /* time id = the frame's position in the visible window:
+                                     sinks 0..S-1, then the kept history and the chunk up to
+                                     W-1 (the slot-order reading of [P4] §机制三)        */
 
 typedef struct rkv_ctx* rkv_handle;
 
@@ -55,7 +58,10 @@ typedef struct rkv_ctx* rkv_handle;
  *  cache size local_attn_size x tokens per frame), of which the first
  *  `sink_frames` frames ever written are never evicted ([P1] §Attention Sink sink_size;
  *  [P4] §机制一 reference-view sinks). `tokens_per_frame` = T; `rope_mode` is
- *  RKV_ROPE_ABSOLUTE or RKV_ROPE_RELATIVE ([P3] §改造③ start_frame; [P4] §机制三).
+ *  RKV_ROPE_ABSOLUTE, RKV_ROPE_RELATIVE or RKV_ROPE_RELATIVE_SLOTS ([P3] §改造③
+ *  start_frame; [P4] §机制三). The two relative modes agree except on the sink frames
+ *  once older non-sink frames have been evicted: clamped re-basing gives such sinks id 0,
+ *  slot order gives sink f id f.
  *  Device memory per layer (library-owned, freed by rkv_destroy, zero-filled):
  *  raw K and V rings [H][window*T][d], a rotated-K ring plus chunk area
  *  [H][(2*window - sink)*T][d] and a rotated-Q staging area [H][(window-sink)*T][d].
@@ -178,8 +184,10 @@ int rkv_cross_attention(rkv_handle h, int layer, const void* q, void* out, int n
  * rkv_rope_apply - rotate x [n_frames*T, H, d] in place with the handle's 3D
  *  RoPE. Absolute mode: t = frame index ([P3] §改造③ rope_apply(..., start_frame)).
  *  Relative mode: t = clamp(f - (window_end_frame - window_frames), 0, W-1),
- *  window_end_frame = one past the last frame of the window ([P4] §机制三);
- *  ignored in absolute mode. fp32 arithmetic, bf16 round-to-nearest-even out.
+ *  window_end_frame = one past the last frame of the window ([P4] §机制三).
+ *  Slot-order mode: t = f for a sink frame (f < sink_frames), otherwise
+ *  f - max(0, window_end_frame - window_frames), then clamped to [0, W-1] (the
+ *  frame's position in that window). window_end_frame is ignored in absolute mode. fp32 arithmetic, bf16 round-to-nearest-even out.
  *  Errors: RKV_ERR_ARG, RKV_ERR_STATE, RKV_ERR_UNSUPPORTED, RKV_ERR_CUDA.
  */
 int rkv_rope_apply(rkv_handle h, void* x, int n_frames, int start_frame,

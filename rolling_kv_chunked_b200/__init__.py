@@ -27,6 +27,7 @@ ERR_STATE = 7
 
 ROPE_ABSOLUTE = 0
 ROPE_RELATIVE = 1
+ROPE_RELATIVE_SLOTS = 2
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is not built; run `python rolling_kv_chunked_b200/build.py`")

@@ -157,7 +157,7 @@ FrameRunParams base_runs(const rkv_ctx* h) {
   p.pairs_h = h->ph;
   p.pairs_w = h->pw;
   p.t_lo = 0;
-  p.t_hi = h->mode == RKV_ROPE_RELATIVE ? h->W - 1 : kTimeTable - 1;
+  p.t_hi = h->mode == RKV_ROPE_ABSOLUTE ? kTimeTable - 1 : h->W - 1;
   p.tab_t = h->tab_t;
   p.tab_h = h->tab_h;
   p.tab_w = h->tab_w;
@@ -273,7 +273,8 @@ RKV_API int rkv_create(int layers, int H, int d, int tokens_per_frame, int windo
   if (layers <= 0 || H <= 0 || d <= 0 || tokens_per_frame <= 0 || window_frames <= 0 || sink_frames < 0 ||
       sink_frames >= window_frames)
     return RKV_ERR_ARG;
-  if (rope_mode != RKV_ROPE_ABSOLUTE && rope_mode != RKV_ROPE_RELATIVE) return RKV_ERR_ARG;
+  if (rope_mode != RKV_ROPE_ABSOLUTE && rope_mode != RKV_ROPE_RELATIVE && rope_mode != RKV_ROPE_RELATIVE_SLOTS)
+    return RKV_ERR_ARG;
   if (d != kHeadDim || window_frames > 256) return RKV_ERR_UNSUPPORTED;
   const long long ring_rows = static_cast<long long>(window_frames) * tokens_per_frame;
   const long long rot_rows = static_cast<long long>(2 * window_frames - sink_frames) * tokens_per_frame;
@@ -441,7 +442,12 @@ int chunk_attention_impl(rkv_handle h, int layer, const void* q, const void* k, 
   const bool abs_mode = h->mode == RKV_ROPE_ABSOLUTE;
   const int C = n_frames, T = h->T, W = h->W;
   if (abs_mode && start_frame + C > kTimeTable) return RKV_ERR_UNSUPPORTED;
-  const long long base = static_cast<long long>(start_frame) + C - W;  // relative re-basing origin
+  // relative re-basing origin: the chunk's last frame gets id W-1 (clamped mode), or
+  // the number of non-sink frames evicted so far (slot-order mode, where ids are
+  // positions in the visible window and sinks keep their own frame index)
+  const bool slot_mode = h->mode == RKV_ROPE_RELATIVE_SLOTS;
+  const long long end = static_cast<long long>(start_frame) + C;
+  const long long base = slot_mode ? std::max<long long>(0, end - W) : end - W;
   const int t_chunk0 = abs_mode ? start_frame : static_cast<int>(start_frame - base);
   const long long ring_rows = static_cast<long long>(W) * T;
   const long long rot_rows = static_cast<long long>(2 * W - h->S) * T;
@@ -481,7 +487,8 @@ int chunk_attention_impl(rkv_handle h, int layer, const void* q, const void* k, 
       r.dst = L.rotk;
       r.src_tok0 = r.dst_tok0 = segs[i].first * T;
       r.n_tok = segs[i].n * T;
-      r.t0 = static_cast<int>(segs[i].frame0 - base);  // clamped to [0, W-1] in the kernel
+      const bool sinks = segs[i].frame0 < h->S;  // the sink segment starts at frame 0
+      r.t0 = static_cast<int>(slot_mode && sinks ? segs[i].frame0 : segs[i].frame0 - base);  // clamped in the kernel
       r.rotate = 1;
       add_run(p, r);
       max_tok = std::max(max_tok, r.n_tok);
@@ -676,14 +683,29 @@ RKV_API int rkv_rope_apply(rkv_handle h, void* x, int n_frames, int start_frame,
   r.dst = static_cast<uint16_t*>(x);
   r.n_tok = n_frames * h->T;
   r.rotate = 1;
+  auto clamp30 = [](long long t) { return static_cast<int>(std::max<long long>(std::min<long long>(t, 1 << 30), -(1 << 30))); };
   if (abs_mode) {
     r.t0 = start_frame;
+  } else if (h->mode == RKV_ROPE_RELATIVE) {
+    r.t0 = clamp30(static_cast<long long>(start_frame) - (static_cast<long long>(window_end_frame) - h->W));
   } else {
-    const long long t0 = static_cast<long long>(start_frame) - (static_cast<long long>(window_end_frame) - h->W);
-    r.t0 = static_cast<int>(std::max<long long>(std::min<long long>(t0, 1 << 30), -(1 << 30)));
+    // slot order: sink frames keep their index, later frames lose the evicted count
+    const long long evicted = std::max<long long>(0, static_cast<long long>(window_end_frame) - h->W);
+    const int n_sink = std::max(0, std::min(n_frames, h->S - start_frame));
+    if (n_sink > 0) {
+      FrameRun rs = r;
+      rs.n_tok = n_sink * h->T;
+      rs.t0 = start_frame;
+      add_run(p, rs);
+      r.src_tok0 = r.dst_tok0 = rs.n_tok;
+      r.n_tok -= rs.n_tok;
+    }
+    r.t0 = clamp30(static_cast<long long>(start_frame) + n_sink - evicted);
+    if (r.n_tok == 0) return cuda_rc(rkv::launch_frame_runs(p, n_sink * h->T, static_cast<cudaStream_t>(stream)));
   }
+  const int max_tok = std::max(r.n_tok, p.n_runs ? p.run[0].n_tok : 0);
   add_run(p, r);
-  return cuda_rc(rkv::launch_frame_runs(p, r.n_tok, static_cast<cudaStream_t>(stream)));
+  return cuda_rc(rkv::launch_frame_runs(p, max_tok, static_cast<cudaStream_t>(stream)));
 }
 
 RKV_API int rkv_flow_x0_renoise(const void* xt, const void* v, const void* eps, double sigma, double sigma_next,

@@ -93,6 +93,8 @@ def test_create_rejects_bad_arguments_before_touching_the_device():
     assert lib.rkv_create(1, 2, 128, 16, 6, 6, 0, ctypes.byref(h)) == rkv.ERR_ARG           # sink >= window
     assert lib.rkv_create(0, 2, 128, 16, 6, 2, 0, ctypes.byref(h)) == rkv.ERR_ARG
     assert lib.rkv_create(1, 2, 128, 16, 6, 2, 7, ctypes.byref(h)) == rkv.ERR_ARG           # rope mode
+    assert lib.rkv_create(1, 2, 128, 16, 6, 2, 3, ctypes.byref(h)) == rkv.ERR_ARG
+    assert lib.rkv_create(1, 2, 128, 16, 6, 2, -1, ctypes.byref(h)) == rkv.ERR_ARG
     assert lib.rkv_create(1, 2, 128, 16, 6, 2, 0, None) == rkv.ERR_ARG
     assert h.value is None
 

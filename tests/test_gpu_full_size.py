@@ -19,13 +19,15 @@ torch = pytest.importorskip("torch")
 if not torch.cuda.is_available():
     pytest.skip("no CUDA device", allow_module_level=True)
 
-ABS, REL = OracleLayer.ABSOLUTE, OracleLayer.RELATIVE
+ABS, REL, SLOTS = OracleLayer.ABSOLUTE, OracleLayer.RELATIVE, OracleLayer.RELATIVE_SLOTS
 
 FULL = [
     # five reference frames become the sinks; evictions start at chunk 5; chunk 6 wraps the ring
     (Config("abot", 20, H=24, grid_h=22, grid_w=40, C=3, W=21, S=5, rope_mode=REL, refs=5, chunks=7, reads=1), (5, 6)),
     # chunk 1 straddles the sink boundary; evictions start at chunk 4
     (Config("480p", 21, H=40, grid_h=30, grid_w=52, C=4, W=18, S=6, rope_mode=ABS, chunks=6, reads=1), (1, 4, 5)),
+    # the ABot shape with slot-order relative ids (the five reference sinks keep ids 0..4)
+    (Config("abot-slots", 23, H=24, grid_h=22, grid_w=40, C=3, W=21, S=5, rope_mode=SLOTS, refs=5, chunks=7, reads=1), (6,)),
     (Config("720p", 22, H=40, grid_h=45, grid_w=80, C=4, W=18, S=6, rope_mode=ABS, chunks=5, reads=1), (4,)),
 ]
 

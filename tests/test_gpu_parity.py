@@ -25,7 +25,7 @@ if not torch.cuda.is_available():
 
 import rolling_kv_chunked_b200 as rkv  # noqa: E402
 
-ABS, REL = OracleLayer.ABSOLUTE, OracleLayer.RELATIVE
+ABS, REL, SLOTS = OracleLayer.ABSOLUTE, OracleLayer.RELATIVE, OracleLayer.RELATIVE_SLOTS
 
 
 def _dev_bits(key, n):
@@ -58,14 +58,15 @@ def test_flow_x0_renoise_bit_exact(n):
             assert np.array_equal(to_bits(xn), rxn), (n, s)
 
 
-@pytest.mark.parametrize("mode", [ABS, REL])
+@pytest.mark.parametrize("mode", [ABS, REL, SLOTS])
 def test_rope_apply_within_one_ulp(mode):
     H, gh, gw, W, n_frames = 3, 6, 7, 9, 4
     T = gh * gw
     h = rkv.RollingKV(1, H, 128, T, W, 2, mode)
     h.set_rope_grid(gh, gw)
     orc = OracleLayer(H, 128, T, gh, gw, W, 2, mode)
-    for start, wend in [(0, 4), (5, 9), (37, 41), (200, 300)]:
+    # (0, 4) and (1, 4) start among the two sinks (split runs in slot-order mode)
+    for start, wend in [(0, 4), (1, 4), (5, 9), (37, 41), (200, 300)]:
         x = _dev_bits(synth.stream_key(1, start), n_frames * T * H * 128).view(n_frames * T, H, 128)
         xb = to_bits(x)
         h.rope_apply(x, n_frames, start, wend)
@@ -86,6 +87,9 @@ SMALL = [
     Config("two-cta", 5, H=2, grid_h=10, grid_w=20, C=2, W=5, S=1, rope_mode=ABS, chunks=6, reads=1),
     Config("straddle", 6, H=2, grid_h=4, grid_w=6, C=4, W=18, S=6, rope_mode=ABS, chunks=8, reads=1),
     Config("no-sink", 7, H=1, grid_h=3, grid_w=5, C=1, W=4, S=0, rope_mode=REL, chunks=9, reads=1),
+    Config("tiny-slots-refs", 8, H=2, grid_h=4, grid_w=4, C=2, W=6, S=2, rope_mode=SLOTS, refs=2, chunks=10),
+    Config("ragged-slots", 9, H=3, grid_h=8, grid_w=10, C=3, W=7, S=2, rope_mode=SLOTS, refs=1, chunks=8, reads=2),
+    Config("straddle-slots", 10, H=2, grid_h=4, grid_w=6, C=4, W=18, S=6, rope_mode=SLOTS, chunks=8, reads=1),
 ]
 
 
