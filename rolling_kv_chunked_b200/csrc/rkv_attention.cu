@@ -26,12 +26,14 @@
 // product straight from TMEM. MMA issue order per key tile j:
 //   S0(j) = Q0 K_j^T, PV1(j-1), S1(j) = Q1 K_j^T, PV0(j)
 // so that while one softmax warpgroup works on its tile the tensor core runs the
-// other tile's products. Online softmax in the log2 domain with a lazy rescale
-// (O is rescaled only when a row maximum grows by more than 2^8). Each softmax thread
-// reads its S row twice from TMEM (once for the maximum, then 64 columns at a time for
-// the exponentials), which keeps the warpgroups within their register budget without
-// spills; exponentials run on the special-function unit, one pair in eight on the FMA
-// pipe as a polynomial, and P is rounded to bf16 with integer operations.
+// other tile's products. Online softmax in the log2 domain against a running reference:
+// each thread reads its S row once (64 columns at a time) and forms the numerators
+// 2^(s/sqrt(d) log2 e - reference) directly; the tile's numerator sum both feeds the row
+// sum and bounds the tile's largest numerator, so the reference moves (and O is rescaled,
+// at the start of the next tile) only when that sum exceeds 2^8, and a sum above 2^64
+// sends the warp to an exact path that takes the row maximum first (always used for the
+// first tile). Exponentials run on the special-function unit, one pair in eight on the
+// FMA pipe as a polynomial; P is rounded to bf16 (nearest even) in pairs.
 //
 // Every mbarrier wait is bounded in wall time; on expiry the kernel records
 // kStatusTimeout in the status word, stops issuing work, waits (bounded) for the
@@ -56,8 +58,9 @@ constexpr int kSmemV = 4 * kTile;         // V stage 0, 1
 constexpr int kSmemBar = 6 * kTile;
 constexpr int kSmemBytes = 6 * kTile + 256 + 1024;  // tiles + barriers + alignment slack
 constexpr unsigned long long kDrainNs = 2000000000ull;
-constexpr float kLazyRescale = 8.0f;  // move the reference only when a maximum grows by more than 2^8
-constexpr float kRefSlack = 64.0f;    // largest accepted x = s * sl2 - reference in the one-pass path
+constexpr float kLazyRescale = 8.0f;    // exact path: move the reference when a maximum grows by > 2^8
+constexpr float kLazySum = 256.0f;      // one-pass path: move the reference when a tile sum exceeds 2^8
+constexpr float kSumSlack = 18446744073709551616.0f;  // 2^64: largest accepted one-pass tile sum
 
 enum : int {
   kBarQ = 0,
@@ -122,11 +125,12 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // f = x - r in [-1/2, 1/2], 2^f by a degree-3 polynomial (max relative error 7.5e-5,
 // coefficients fitted for minimal relative error by rolling_kv_chunked_b200/exp2_poly.py),
 // then r is added to the exponent field (the bits of 1.5*2^23 vanish under << 23).
-// x is clamped at -125 so the result stays a positive normal number.
+// x is clamped to [-125, 126] so the result stays a positive normal number (a score far
+// above the reference then shows up as a huge tile sum, as it does on the other path).
 __device__ __forceinline__ void exp2_poly_x2(uint64_t x2, float& y0, float& y1) {
   float x0, x1;
   ptx::f2_unpack(x2, x0, x1);
-  const uint64_t x = ptx::f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+  const uint64_t x = ptx::f2_pack(fminf(fmaxf(x0, -125.0f), 126.0f), fminf(fmaxf(x1, -125.0f), 126.0f));
   const uint64_t magic = ptx::f2_pack(12582912.0f, 12582912.0f);
   const uint64_t neg_magic = ptx::f2_pack(-12582912.0f, -12582912.0f);
   const uint64_t neg_one = ptx::f2_pack(-1.0f, -1.0f);
@@ -175,26 +179,32 @@ __device__ __forceinline__ void softmax_half(const uint32_t* sh, uint64_t c2, ui
 }
 
 // The same numerators for a whole 64-key half computed against the running reference
-// (nm2 = -m) without storing them: packed pairs go to pk[0..31], and mx[0], mx[1] track the
-// largest x = s * sl2 - m, so that the caller can check the reference afterwards.
+// (nm2 = -m) without storing them: packed pairs go to pk[0..31], so that the caller can
+// check the tile sum before S is overwritten.
 template <bool kPoly>
 __device__ __forceinline__ void numerators_half(const uint32_t* sh, uint64_t c2, uint64_t nm2, uint32_t* pk,
-                                                uint64_t (&acc)[4], float (&mx)[2]) {
+                                                uint64_t (&acc)[4]) {
 #pragma unroll
   for (int k = 0; k < kBN / 4; ++k) {
     const uint64_t x = ptx::f2_fma(ptx::f2_pack(__uint_as_float(sh[2 * k]), __uint_as_float(sh[2 * k + 1])), c2, nm2);
-    float x0, x1, a, b;
-    ptx::f2_unpack(x, x0, x1);
-    mx[k & 1] = ptx::fmax3(mx[k & 1], x0, x1);
+    float a, b;
     if (kPoly && (k & 7) < kPolyPairs) {
       exp2_poly_x2(x, a, b);
     } else {
+      float x0, x1;
+      ptx::f2_unpack(x, x0, x1);
       a = ptx::ex2(x0);
       b = ptx::ex2(x1);
     }
     acc[k & 3] = ptx::f2_add(acc[k & 3], ptx::f2_pack(a, b));
     pk[k] = pack_bf16x2(a, b);
   }
+}
+
+__device__ __forceinline__ float lg2_approx(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // O (this thread's row, 128 fp32 TMEM columns at tO) *= f
@@ -351,14 +361,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m_used = -INFINITY;  // reference of the numerators, log2 units: p = 2^(s * sl2 - m_used)
     float l = 0.f;             // row sum of the numerators, in the scale of the reference
     float pend = 1.0f;         // change of reference decided on the previous tile, not yet applied
+    // the ragged last tile of each key segment: its index in the stream and its valid keys
+    int rag_j[kMaxSegs], rag_v[kMaxSegs];
+    {
+      int first = 0;
+#pragma unroll
+      for (int sg = 0; sg < kMaxSegs; ++sg) {
+        rag_j[sg] = -1;
+        rag_v[sg] = kBN;
+        if (sg < p.n_segs) {
+          const int nt = (p.seg[sg].n_rows + kBN - 1) / kBN;
+          rag_j[sg] = first + nt - 1;
+          rag_v[sg] = p.seg[sg].n_rows - (nt - 1) * kBN;
+          first += nt;
+        }
+      }
+    }
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
       ok = ptx::mbar_wait(&bars[kBarSFull + wg], j & 1, limit);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       ptx::tc_fence_after();
-      int src, krow, vrow, valid;
-      tile_of(p, j, src, krow, vrow, valid);
+      int valid = kBN;
+#pragma unroll
+      for (int sg = 0; sg < kMaxSegs; ++sg)
+        if (j == rag_j[sg]) valid = rag_v[sg];
       // S(j) complete implies PV(j-1) complete: O now holds every product in the previous
       // reference's scale, so a pending change applies to O and l together
       if (__any_sync(0xffffffffu, pend != 1.0f)) scale_o(tO, pend);
@@ -366,12 +394,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       pend = 1.0f;
       bool stored = false;
       if (j > 0) {
-        // one pass against the running reference; the tile maximum comes out of the same
-        // pass (on the integer ALU, under the special-function-unit work) instead of a
-        // separate pass before it
+        // one pass against the running reference
         const uint64_t nm2 = ptx::f2_pack(-m_used, -m_used);
         uint64_t acc[4] = {0, 0, 0, 0};
-        float mx2[2] = {-INFINITY, -INFINITY};
         uint32_t pk[kBN / 2];
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
@@ -381,23 +406,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < kBN / 2; ++i)
               if (64 * hh + i >= valid) sh[i] = 0xff800000u;
-            numerators_half<false>(sh, c2, nm2, pk + 32 * hh, acc, mx2);
+            numerators_half<false>(sh, c2, nm2, pk + 32 * hh, acc);
           } else {
-            numerators_half<true>(sh, c2, nm2, pk + 32 * hh, acc, mx2);
+            numerators_half<true>(sh, c2, nm2, pk + 32 * hh, acc);
           }
         }
-        const float mx = fmaxf(mx2[0], mx2[1]);
-        // numerators up to 2^64 are exact in bf16 / fp32 range and keep O finite; a score
-        // further above the reference sends the whole warp to the exact path below, which
-        // recomputes the tile from S (not overwritten yet)
-        if (!__any_sync(0xffffffffu, mx > kRefSlack)) {
-          float rs[4];
-          ptx::f2_unpack(ptx::f2_add(acc[0], acc[1]), rs[0], rs[1]);
-          ptx::f2_unpack(ptx::f2_add(acc[2], acc[3]), rs[2], rs[3]);
-          l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
-          if (mx > kLazyRescale) {  // move the reference to this tile's maximum from the next tile on
-            pend = ptx::ex2(-mx);
-            m_used += mx;
+        float rs[4];
+        ptx::f2_unpack(ptx::f2_add(acc[0], acc[1]), rs[0], rs[1]);
+        ptx::f2_unpack(ptx::f2_add(acc[2], acc[3]), rs[2], rs[3]);
+        const float lt = (rs[0] + rs[1]) + (rs[2] + rs[3]);
+        // the tile's numerator sum bounds its largest numerator: 2^max <= lt <= 128 * 2^max.
+        // A sum above 2^64 (or not a number) sends the warp to the exact path below.
+        if (!__any_sync(0xffffffffu, !(lt <= kSumSlack))) {
+          l += lt;
+          if (lt > kLazySum) {  // move the reference up by log2(lt) from the next tile on
+            const float sh = lg2_approx(lt);
+            pend = ptx::ex2(-sh);
+            m_used += sh;
           }
           ptx::tmem_st64(tS, pk);
           stored = true;

@@ -147,6 +147,52 @@ def test_outputs_are_deterministic():
     h.close()
 
 
+@pytest.mark.parametrize("sink_score", [-2000.0, -150.0, 400.0])
+@pytest.mark.parametrize("mode", [ABS, REL])
+def test_score_jumps_between_key_tiles(sink_score, mode):
+    """The sink frame fills the first key tile with scores far below (or above) the rest.
+    -2000: the later tiles' numerators overflow against the first tile's reference, so the
+    exact path (maximum first) must take over; -150: the reference moves lazily (tile sums
+    near 2^19); +400: the first tile dominates and the later ones underflow. Queries share
+    one direction u on the lowest-frequency rotary pairs (near-zero rotation at these
+    positions), so q.k_sink stays close to the chosen score whatever the positions."""
+    H, gh, gw, W, S, C = 2, 8, 16, 4, 1, 1
+    T = gh * gw
+    rng = np.random.default_rng(int(abs(sink_score)) + 7 * mode)
+    low = [p for p in range(64) if 17 <= p < 22 or 38 <= p < 43 or 59 <= p < 64]
+    dims = np.array([2 * p + e for p in low for e in (0, 1)])
+    u = np.zeros((H, 128))
+    u[:, dims] = rng.standard_normal((H, len(dims)))
+    qf = np.broadcast_to(u, (C * T, H, 128)).copy()
+    ksink = np.broadcast_to(sink_score * u / np.sum(u * u, axis=1, keepdims=True), (T, H, 128))
+
+    def bits(x):
+        return bf16.from_f64(np.asarray(x, dtype=np.float64))
+
+    def dev(b):
+        return torch.from_numpy(b.view(np.int16)).cuda().view(torch.bfloat16)
+
+    h = rkv.RollingKV(1, H, 128, T, W, S, mode)
+    h.set_rope_grid(gh, gw)
+    orc = OracleLayer(H, 128, T, gh, gw, W, S, mode)
+    kb, vb = bits(ksink), bits(rng.standard_normal((T, H, 128)))
+    h.write_chunk(0, dev(kb), dev(vb), 1, 0)
+    orc.write_chunk(kb, vb, 1, 0)
+    qb = bits(qf)
+    for f0 in range(1, 6):
+        kb, vb = bits(rng.standard_normal((T, H, 128))), bits(rng.standard_normal((T, H, 128)))
+        out = torch.empty((C * T, H, 128), dtype=torch.bfloat16, device="cuda")
+        for commit in (False, True):
+            h.chunk_attention(0, dev(qb), dev(kb), dev(vb), out, C, f0, commit)
+            torch.cuda.synchronize()
+            ref = orc.chunk_attention(qb, kb, vb, C, f0, commit)
+            got = to_bits(out)
+            assert np.all(np.isfinite(bf16.to_f64(got)))
+            assert_close(got, ref, f"sink score {sink_score} frame {f0} commit {commit}")
+    assert h.poll_device_status() == rkv.OK
+    h.close()
+
+
 def test_host_errors_launch_nothing():
     cfg = Config("err", 10, H=2, grid_h=4, grid_w=4, C=2, W=6, S=2, rope_mode=ABS)
     h = rkv.RollingKV(1, cfg.H, 128, cfg.T, cfg.W, cfg.S, cfg.rope_mode)
