@@ -15,13 +15,7 @@
 // the cross-attention over the cached text K/V: one key segment, queries read token-major
 // straight from the caller's buffer, no rotation.
 //
-// Work is split into units: one head x 256 query rows (two 128-row tiles Q0, Q1) against
-// the whole key stream. Either one CTA runs one unit, or (when the units outnumber the SMs
-// and would leave a partial last wave) one persistent CTA per SM runs an equal share of all
-// (unit, key tile) pairs in order ("stream-K"): a unit cut at a CTA boundary is computed in
-// two parts, each part publishes its unnormalised O, reference and row sum, and the part
-// that arrives second (counted per warp with an atomic, no waiting) merges both and stores
-// the rows. Structure of one CTA:
+// Structure of one CTA (one head, 256 query rows = two 128-row tiles Q0, Q1):
 //   warps 0-3  softmax for Q0 (one thread per query row = TMEM lane)
 //   warps 4-7  softmax for Q1
 //   warp 8     TMA producer: Q0/Q1 once, then K and V tiles (128 keys) into a
@@ -78,8 +72,7 @@ enum : int {
   kBarPFull = 11,  // +tile
   kBarODone = 13,
   kBarDrain = 14,
-  kBarQEmpty = 15,  // every S product of the current unit has completed
-  kNumBars = 16
+  kNumBars = 15
 };
 
 // TMEM column of the S / P tile and of the O accumulator of query tile t (0 or 1).
@@ -226,26 +219,6 @@ __device__ __forceinline__ void scale_o(uint32_t tO, float f) {
   }
 }
 
-// The (unit, tile) pairs this CTA processes: [g0, g1) in the order unit-major, tile-minor.
-__device__ __forceinline__ void cta_range(const AttnParams& p, int n_units, long long& g0, long long& g1) {
-  const long long nt = p.n_tiles;
-  if (p.sk_ctas > 0) {
-    const long long total = static_cast<long long>(n_units) * nt;
-    g0 = total * blockIdx.x / p.sk_ctas;
-    g1 = total * (blockIdx.x + 1) / p.sk_ctas;
-  } else {
-    g0 = static_cast<long long>(blockIdx.x) * nt;
-    g1 = g0 + nt;
-  }
-}
-
-// The run of tiles [a, b) of unit u that starts at pair g (g < g1).
-__device__ __forceinline__ void unit_run(const AttnParams& p, long long g, long long g1, int& u, int& a, int& b) {
-  u = static_cast<int>(g / p.n_tiles);
-  a = static_cast<int>(g - static_cast<long long>(u) * p.n_tiles);
-  b = static_cast<int>(min(static_cast<long long>(p.n_tiles), a + (g1 - g)));
-}
-
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                            const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_vn,
@@ -253,18 +226,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSmemBar);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 24);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int n_qblocks = (p.Lq + 2 * kBM - 1) / (2 * kBM);
-  long long g0, g1;
-  cta_range(p, n_qblocks * p.H, g0, g1);
+  const int head = blockIdx.y;
+  const int m0 = blockIdx.x * (2 * kBM);
   const unsigned long long limit = p.wait_limit_ns;
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(&bars[kBarQ], 1);
-    ptx::mbar_init(&bars[kBarQEmpty], 1);
     for (int s = 0; s < 2; ++s) {
       ptx::mbar_init(&bars[kBarKFull + s], 1);
       ptx::mbar_init(&bars[kBarKEmpty + s], 1);
@@ -285,6 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const int n_tiles = p.n_tiles;
 
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
@@ -293,50 +265,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::prefetch_tmap(&tm_k);
       ptx::prefetch_tmap(&tm_vc);
       ptx::prefetch_tmap(&tm_vn);
+      ptx::mbar_arrive_expect_tx(&bars[kBarQ], 2 * kTile);
+      for (int t = 0; t < 2; ++t)
+        for (int c = 0; c < 2; ++c)
+          if (p.q_token_major)
+            ptx::tma_load_3d(smem + kSmemQ + t * kTile + c * kSlab, &tm_q, &bars[kBarQ], c * 64, head, m0 + t * kBM);
+          else
+            ptx::tma_load_3d(smem + kSmemQ + t * kTile + c * kSlab, &tm_q, &bars[kBarQ], c * 64, m0 + t * kBM, head);
       bool ok = true;
-      int gk = 0;                // key / value tiles issued by this CTA (all units)
-      int nq = 0, nk = 0, nv = 0;  // Q / K / V loads issued
-      for (long long g = g0; ok && g < g1;) {
-        int u, a, b;
-        unit_run(p, g, g1, u, a, b);
-        g += b - a;
-        const int head = u / n_qblocks;
-        const int m0 = (u - head * n_qblocks) * (2 * kBM);
-        // the previous unit's S products must have read the Q tiles
-        if (nq > 0 && !ptx::mbar_wait(&bars[kBarQEmpty], (nq - 1) & 1, limit)) { ok = false; break; }
-        ptx::mbar_arrive_expect_tx(&bars[kBarQ], 2 * kTile);
-        for (int t = 0; t < 2; ++t)
-          for (int c = 0; c < 2; ++c)
-            if (p.q_token_major)
-              ptx::tma_load_3d(smem + kSmemQ + t * kTile + c * kSlab, &tm_q, &bars[kBarQ], c * 64, head, m0 + t * kBM);
-            else
-              ptx::tma_load_3d(smem + kSmemQ + t * kTile + c * kSlab, &tm_q, &bars[kBarQ], c * 64, m0 + t * kBM, head);
-        ++nq;
-        for (int j = a; j < b; ++j, ++gk) {
-          const int s = gk & 1;
-          int src, krow, vrow, valid;
-          tile_of(p, j, src, krow, vrow, valid);
-          if (gk >= 2 && !ptx::mbar_wait(&bars[kBarKEmpty + s], ((gk - 2) >> 1) & 1, limit)) { ok = false; break; }
-          ptx::mbar_arrive_expect_tx(&bars[kBarKFull + s], kTile);
-          for (int c = 0; c < 2; ++c)
-            ptx::tma_load_3d(smem + kSmemK + s * kTile + c * kSlab, &tm_k, &bars[kBarKFull + s], c * 64, krow, head);
-          nk = gk + 1;
-          if (gk >= 2 && !ptx::mbar_wait(&bars[kBarVEmpty + s], ((gk - 2) >> 1) & 1, limit)) { ok = false; break; }
-          ptx::mbar_arrive_expect_tx(&bars[kBarVFull + s], kTile);
-          for (int c = 0; c < 2; ++c) {
-            if (src == 0)
-              ptx::tma_load_3d(smem + kSmemV + s * kTile + c * kSlab, &tm_vc, &bars[kBarVFull + s], c * 64, vrow, head);
-            else
-              ptx::tma_load_3d(smem + kSmemV + s * kTile + c * kSlab, &tm_vn, &bars[kBarVFull + s], c * 64, head, vrow);
-          }
-          nv = gk + 1;
+      int nk = 0, nv = 0;
+      for (int j = 0; j < n_tiles; ++j) {
+        const int s = j & 1;
+        int src, krow, vrow, valid;
+        tile_of(p, j, src, krow, vrow, valid);
+        if (j >= 2 && !ptx::mbar_wait(&bars[kBarKEmpty + s], ((j - 2) >> 1) & 1, limit)) { ok = false; break; }
+        ptx::mbar_arrive_expect_tx(&bars[kBarKFull + s], kTile);
+        for (int c = 0; c < 2; ++c)
+          ptx::tma_load_3d(smem + kSmemK + s * kTile + c * kSlab, &tm_k, &bars[kBarKFull + s], c * 64, krow, head);
+        nk = j + 1;
+        if (j >= 2 && !ptx::mbar_wait(&bars[kBarVEmpty + s], ((j - 2) >> 1) & 1, limit)) { ok = false; break; }
+        ptx::mbar_arrive_expect_tx(&bars[kBarVFull + s], kTile);
+        for (int c = 0; c < 2; ++c) {
+          if (src == 0)
+            ptx::tma_load_3d(smem + kSmemV + s * kTile + c * kSlab, &tm_vc, &bars[kBarVFull + s], c * 64, vrow, head);
+          else
+            ptx::tma_load_3d(smem + kSmemV + s * kTile + c * kSlab, &tm_vn, &bars[kBarVFull + s], c * 64, head, vrow);
         }
+        nv = j + 1;
       }
       if (!ok) atomicOr(p.status, kStatusTimeout);
       // every copy issued must land before the CTA may exit
-      if (nq > 0) ptx::mbar_wait(&bars[kBarQ], (nq - 1) & 1, kDrainNs);
-      for (int t = (nk > 2 ? nk - 2 : 0); t < nk; ++t) ptx::mbar_wait(&bars[kBarKFull + (t & 1)], (t >> 1) & 1, kDrainNs);
-      for (int t = (nv > 2 ? nv - 2 : 0); t < nv; ++t) ptx::mbar_wait(&bars[kBarVFull + (t & 1)], (t >> 1) & 1, kDrainNs);
+      ptx::mbar_wait(&bars[kBarQ], 0, kDrainNs);
+      for (int j = (nk > 2 ? nk - 2 : 0); j < nk; ++j) ptx::mbar_wait(&bars[kBarKFull + (j & 1)], (j >> 1) & 1, kDrainNs);
+      for (int j = (nv > 2 ? nv - 2 : 0); j < nv; ++j) ptx::mbar_wait(&bars[kBarVFull + (j & 1)], (j >> 1) & 1, kDrainNs);
     }
     __syncwarp();
   } else if (warp == 9) {
@@ -345,56 +306,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t q_addr[2] = {ptx::smem_u32(smem + kSmemQ), ptx::smem_u32(smem + kSmemQ + kTile)};
       const uint32_t k_addr = ptx::smem_u32(smem + kSmemK);
       const uint32_t v_addr = ptx::smem_u32(smem + kSmemV);
+      bool ok = ptx::mbar_wait(&bars[kBarQ], 0, limit);
 
       auto issue_s = [&](int t, uint32_t kt) {
 #pragma unroll
         for (int kk = 0; kk < kHeadDim / 16; ++kk)
           ptx::mma_ss(tmem + col_s(t), desc_kmajor(q_addr[t], kk), desc_kmajor(kt, kk), kIdescS, kk > 0 ? 1u : 0u);
       };
-      // O_t += P_t V for the CTA's tile number gt (first: the unit's first tile, O starts from
-      // zero); returns false if a wait expired
-      auto issue_pv = [&](int t, int gt, bool first) -> bool {
-        if (!ptx::mbar_wait(&bars[kBarPFull + t], gt & 1, limit)) return false;
-        if (!ptx::mbar_wait(&bars[kBarVFull + (gt & 1)], (gt >> 1) & 1, limit)) return false;
+      // O_t += P_t(jj) V(jj); returns false if a wait expired
+      auto issue_pv = [&](int t, int jj) -> bool {
+        if (!ptx::mbar_wait(&bars[kBarPFull + t], jj & 1, limit)) return false;
+        if (!ptx::mbar_wait(&bars[kBarVFull + (jj & 1)], (jj >> 1) & 1, limit)) return false;
         ptx::tc_fence_after();
-        const uint32_t vt = v_addr + (gt & 1) * kTile;
+        const uint32_t vt = v_addr + (jj & 1) * kTile;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
           ptx::mma_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8, desc_v(vt, kk), kIdescPV,
-                      (!first || kk > 0) ? 1u : 0u);
-        if (t == 1) ptx::mma_commit(&bars[kBarVEmpty + (gt & 1)]);
+                      (jj > 0 || kk > 0) ? 1u : 0u);
+        if (t == 1) ptx::mma_commit(&bars[kBarVEmpty + (jj & 1)]);
         return true;
       };
 
-      bool ok = true;
-      int gt0 = 0;  // tiles of the CTA's earlier units
-      int nu = 0;   // units started
-      for (long long g = g0; ok && g < g1; ++nu) {
-        int u, a, b;
-        unit_run(p, g, g1, u, a, b);
-        const int n = b - a;
-        g += n;
-        if (!ptx::mbar_wait(&bars[kBarQ], nu & 1, limit)) { ok = false; break; }
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        const int s = j & 1;
+        if (!ptx::mbar_wait(&bars[kBarKFull + s], (j >> 1) & 1, limit)) { ok = false; break; }
         ptx::tc_fence_after();
-        for (int j = 0; j < n; ++j) {
-          const int gt = gt0 + j;
-          const int s = gt & 1;
-          if (!ptx::mbar_wait(&bars[kBarKFull + s], (gt >> 1) & 1, limit)) { ok = false; break; }
-          ptx::tc_fence_after();
-          const uint32_t kt = k_addr + s * kTile;
-          issue_s(0, kt);
-          ptx::mma_commit(&bars[kBarSFull + 0]);
-          if (j > 0 && !issue_pv(1, gt - 1, j == 1)) { ok = false; break; }
-          issue_s(1, kt);
-          ptx::mma_commit(&bars[kBarSFull + 1]);
-          ptx::mma_commit(&bars[kBarKEmpty + s]);
-          if (j == n - 1) ptx::mma_commit(&bars[kBarQEmpty]);  // the unit's last S products
-          if (!issue_pv(0, gt, j == 0)) { ok = false; break; }
-        }
-        if (ok && !issue_pv(1, gt0 + n - 1, n == 1)) ok = false;
-        if (ok) ptx::mma_commit(&bars[kBarODone]);
-        gt0 += n;
+        const uint32_t kt = k_addr + s * kTile;
+        issue_s(0, kt);
+        ptx::mma_commit(&bars[kBarSFull + 0]);
+        if (j > 0 && !issue_pv(1, j - 1)) { ok = false; break; }
+        issue_s(1, kt);
+        ptx::mma_commit(&bars[kBarSFull + 1]);
+        ptx::mma_commit(&bars[kBarKEmpty + s]);
+        if (!issue_pv(0, j)) { ok = false; break; }
       }
+      if (ok && !issue_pv(1, n_tiles - 1)) ok = false;
+      if (ok) ptx::mma_commit(&bars[kBarODone]);
       if (!ok) atomicOr(p.status, kStatusTimeout);
       // everything issued must complete before TMEM is released
       ptx::mma_commit(&bars[kBarDrain]);
@@ -411,6 +358,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tO = lane_base + col_o(wg);
     const float sl2 = p.scale_log2;
     const uint64_t c2 = ptx::f2_pack(sl2, sl2);
+    float m_used = -INFINITY;  // reference of the numerators, log2 units: p = 2^(s * sl2 - m_used)
+    float l = 0.f;             // row sum of the numerators, in the scale of the reference
+    float pend = 1.0f;         // change of reference decided on the previous tile, not yet applied
     // the ragged last tile of each key segment: its index in the stream and its valid keys
     int rag_j[kMaxSegs], rag_v[kMaxSegs];
     {
@@ -428,250 +378,181 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     bool ok = true;
-    int gt0 = 0;  // tiles of the CTA's earlier units
-    int nu = 0;   // units started
-    for (long long g = g0; ok && g < g1; ++nu) {
-      int u, a, b;
-      unit_run(p, g, g1, u, a, b);
-      const int n = b - a;
-      g += n;
-      float m_used = -INFINITY;  // reference of the numerators, log2 units: p = 2^(s * sl2 - m_used)
-      float m_ol = -INFINITY;    // the reference of the values now in O and l
-      float l = 0.f;             // row sum of the numerators, in the scale of m_ol
-      float pend = 1.0f;         // change of reference decided on the previous tile, not yet applied
-      for (int jl = 0; jl < n; ++jl) {
-        const int j = a + jl;    // tile within the unit's key stream
-        ok = ptx::mbar_wait(&bars[kBarSFull + wg], (gt0 + jl) & 1, limit);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        ptx::tc_fence_after();
-        int valid = kBN;
-#pragma unroll
-        for (int sg = 0; sg < kMaxSegs; ++sg)
-          if (j == rag_j[sg]) valid = rag_v[sg];
-        // S(j) complete implies PV(j-1) complete: O now holds every product in the previous
-        // reference's scale, so a pending change applies to O and l together
-        if (__any_sync(0xffffffffu, pend != 1.0f)) scale_o(tO, pend);
-        l *= pend;
-        pend = 1.0f;
-        m_ol = m_used;
-        bool stored = false;
-        if (jl > 0) {
-          // one pass against the running reference
-          const uint64_t nm2 = ptx::f2_pack(-m_used, -m_used);
-          uint64_t acc[4] = {0, 0, 0, 0};
-          uint32_t pk[kBN / 2];
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            uint32_t sh[kBN / 2];
-            ptx::tmem_ld64(tS + 64 * hh, sh);
-            if (valid < kBN) {
-#pragma unroll
-              for (int i = 0; i < kBN / 2; ++i)
-                if (64 * hh + i >= valid) sh[i] = 0xff800000u;
-              numerators_half<false>(sh, c2, nm2, pk + 32 * hh, acc);
-            } else {
-              numerators_half<true>(sh, c2, nm2, pk + 32 * hh, acc);
-            }
-          }
-          float rs[4];
-          ptx::f2_unpack(ptx::f2_add(acc[0], acc[1]), rs[0], rs[1]);
-          ptx::f2_unpack(ptx::f2_add(acc[2], acc[3]), rs[2], rs[3]);
-          const float lt = (rs[0] + rs[1]) + (rs[2] + rs[3]);
-          // the tile's numerator sum bounds its largest numerator: 2^max <= lt <= 128 * 2^max.
-          // A sum above 2^64 (or not a number) sends the warp to the exact path below.
-          if (!__any_sync(0xffffffffu, !(lt <= kSumSlack))) {
-            l += lt;
-            if (lt > kLazySum) {  // move the reference up by log2(lt) from the next tile on
-              const float sh = lg2_approx(lt);
-              pend = ptx::ex2(-sh);
-              m_used += sh;
-            }
-            ptx::tmem_st64(tS, pk);
-            stored = true;
-          }
-        }
-        if (!stored) {
-          // exact path (the first tile, or a score far above the reference): the row maximum
-          // first, then the numerators
-          float m_tile;
-          {
-            uint32_t sr[kBN];
-            ptx::tmem_ld128(tS, sr);
-            if (valid < kBN) {
-#pragma unroll
-              for (int i = 0; i < kBN; ++i)
-                if (i >= valid) sr[i] = 0xff800000u;
-            }
-            float mq[4];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const uint32_t* t = sr + 32 * c;
-              float m = ptx::fmax3(__uint_as_float(t[0]), __uint_as_float(t[1]), __uint_as_float(t[2]));
-#pragma unroll
-              for (int i = 3; i < 31; i += 2) m = ptx::fmax3(m, __uint_as_float(t[i]), __uint_as_float(t[i + 1]));
-              mq[c] = fmaxf(m, __uint_as_float(t[31]));
-            }
-            m_tile = ptx::fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3])) * sl2;
-          }
-          const bool need = m_tile > m_used + kLazyRescale;
-          float alpha = 1.0f;
-          if (need) {
-            alpha = ptx::ex2(m_used - m_tile);
-            m_used = m_tile;
-          }
-          l *= alpha;
-          if (jl > 0 && __any_sync(0xffffffffu, need)) scale_o(tO, alpha);
-          m_ol = m_used;
-          const uint64_t nm2 = ptx::f2_pack(-m_used, -m_used);
-          uint64_t acc[4] = {0, 0, 0, 0};
-          // reload 64 columns at a time; P of the first half overwrites S columns 0..31,
-          // already read, the second half's loads touch columns 64..127 only
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            uint32_t sh[kBN / 2];
-            ptx::tmem_ld64(tS + 64 * hh, sh);
-            if (valid < kBN) {
-#pragma unroll
-              for (int i = 0; i < kBN / 2; ++i)
-                if (64 * hh + i >= valid) sh[i] = 0xff800000u;
-              softmax_half<false>(sh, c2, nm2, tS + 32 * hh, acc);
-            } else {
-              softmax_half<true>(sh, c2, nm2, tS + 32 * hh, acc);
-            }
-          }
-          float rs[4];
-          ptx::f2_unpack(ptx::f2_add(acc[0], acc[1]), rs[0], rs[1]);
-          ptx::f2_unpack(ptx::f2_add(acc[2], acc[3]), rs[2], rs[3]);
-          l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
-        }
-        ptx::tmem_st_wait();
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(&bars[kBarPFull + wg]);
-      }
-      gt0 += n;
-      if (ok) {
-        ok = ptx::mbar_wait(&bars[kBarODone], nu & 1, limit);
-        ok = __all_sync(0xffffffffu, ok);
-      }
+    for (int j = 0; j < n_tiles; ++j) {
+      ok = ptx::mbar_wait(&bars[kBarSFull + wg], j & 1, limit);
+      ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
-      {
-        ptx::tc_fence_after();
-        const int head = u / n_qblocks;
-        const int m0 = (u - head * n_qblocks) * (2 * kBM);
-        const int ru = wg * kBM + r;  // row within the unit
-        // output = (O * f_own + O_other * f_oth) / (l * f_own + l_other * f_oth)
-        float f_own = 1.0f, f_oth = 0.0f, lsum = l;
-        const float* oth = nullptr;
-        if (a > 0 || b < p.n_tiles) {
-          // a unit cut between two CTAs: publish this part; of the two, the one that arrives
-          // second (decided per warp, i.e. per 32 rows) combines both and stores the rows
-          const int part = a == 0 ? 0 : 1;  // 0: the unit's first tiles, at the end of this CTA's range
-          const int bnd = part == 0 ? static_cast<int>(blockIdx.x) + 1 : static_cast<int>(blockIdx.x);
-          float* mine = p.sk_part + (static_cast<size_t>(bnd) * 2 + part) * kSkPartFloats;
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t v32[32];
-            ptx::tmem_ld32(tO + 32 * c, v32);
-            float4* dst = reinterpret_cast<float4*>(mine + static_cast<size_t>(ru) * kHeadDim + 32 * c);
+      ptx::tc_fence_after();
+      int valid = kBN;
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              __stcg(dst + i, make_float4(__uint_as_float(v32[4 * i]), __uint_as_float(v32[4 * i + 1]),
-                                          __uint_as_float(v32[4 * i + 2]), __uint_as_float(v32[4 * i + 3])));
+      for (int sg = 0; sg < kMaxSegs; ++sg)
+        if (j == rag_j[sg]) valid = rag_v[sg];
+      // S(j) complete implies PV(j-1) complete: O now holds every product in the previous
+      // reference's scale, so a pending change applies to O and l together
+      if (__any_sync(0xffffffffu, pend != 1.0f)) scale_o(tO, pend);
+      l *= pend;
+      pend = 1.0f;
+      bool stored = false;
+      if (j > 0) {
+        // one pass against the running reference
+        const uint64_t nm2 = ptx::f2_pack(-m_used, -m_used);
+        uint64_t acc[4] = {0, 0, 0, 0};
+        uint32_t pk[kBN / 2];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t sh[kBN / 2];
+          ptx::tmem_ld64(tS + 64 * hh, sh);
+          if (valid < kBN) {
+#pragma unroll
+            for (int i = 0; i < kBN / 2; ++i)
+              if (64 * hh + i >= valid) sh[i] = 0xff800000u;
+            numerators_half<false>(sh, c2, nm2, pk + 32 * hh, acc);
+          } else {
+            numerators_half<true>(sh, c2, nm2, pk + 32 * hh, acc);
           }
-          __stcg(mine + 2 * kBM * kHeadDim + ru, m_ol);
-          __stcg(mine + 2 * kBM * (kHeadDim + 1) + ru, l);
-          __threadfence();
-          __syncwarp();
-          unsigned old = 0;
-          if (lane == 0) old = atomicAdd(p.sk_count + bnd * 8 + warp, 1u);
-          old = __shfl_sync(0xffffffffu, old, 0);
-          if ((old & 1u) == 0) continue;  // first to arrive: the other CTA stores these rows
-          __threadfence();
-          oth = p.sk_part + (static_cast<size_t>(bnd) * 2 + (1 - part)) * kSkPartFloats;
-          const float m2 = __ldcg(oth + 2 * kBM * kHeadDim + ru);
-          const float l2 = __ldcg(oth + 2 * kBM * (kHeadDim + 1) + ru);
-          const float mm = fmaxf(m_ol, m2);
-          f_own = ptx::ex2(m_ol - mm);
-          f_oth = ptx::ex2(m2 - mm);
-          lsum = l * f_own + l2 * f_oth;
-          oth += static_cast<size_t>(ru) * kHeadDim;
         }
-        const int row = m0 + ru;
-        const bool live = row < p.Lq;
-        const float inv_l = 1.0f / lsum;
-        const float g_own = f_own * inv_l, g_oth = f_oth * inv_l;
-        const long long base = (static_cast<long long>(row) * p.H + head) * kHeadDim;
-        FlowStep step;
-        step.sigma = p.sigma;
-        step.renoise = p.sigma_next >= 0.0;
-        step.sigma_next = step.renoise ? p.sigma_next : 0.0;
-        step.one_minus_next = __dsub_rn(1.0, step.sigma_next);
+        float rs[4];
+        ptx::f2_unpack(ptx::f2_add(acc[0], acc[1]), rs[0], rs[1]);
+        ptx::f2_unpack(ptx::f2_add(acc[2], acc[3]), rs[2], rs[3]);
+        const float lt = (rs[0] + rs[1]) + (rs[2] + rs[3]);
+        // the tile's numerator sum bounds its largest numerator: 2^max <= lt <= 128 * 2^max.
+        // A sum above 2^64 (or not a number) sends the warp to the exact path below.
+        if (!__any_sync(0xffffffffu, !(lt <= kSumSlack))) {
+          l += lt;
+          if (lt > kLazySum) {  // move the reference up by log2(lt) from the next tile on
+            const float sh = lg2_approx(lt);
+            pend = ptx::ex2(-sh);
+            m_used += sh;
+          }
+          ptx::tmem_st64(tS, pk);
+          stored = true;
+        }
+      }
+      if (!stored) {
+        // exact path (the first tile, or a score far above the reference): the row maximum
+        // first, then the numerators
+        float m_tile;
+        {
+          uint32_t sr[kBN];
+          ptx::tmem_ld128(tS, sr);
+          if (valid < kBN) {
+#pragma unroll
+            for (int i = 0; i < kBN; ++i)
+              if (i >= valid) sr[i] = 0xff800000u;
+          }
+          float mq[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint32_t* t = sr + 32 * c;
+            float m = ptx::fmax3(__uint_as_float(t[0]), __uint_as_float(t[1]), __uint_as_float(t[2]));
+#pragma unroll
+            for (int i = 3; i < 31; i += 2) m = ptx::fmax3(m, __uint_as_float(t[i]), __uint_as_float(t[i + 1]));
+            mq[c] = fmaxf(m, __uint_as_float(t[31]));
+          }
+          m_tile = ptx::fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3])) * sl2;
+        }
+        const bool need = m_tile > m_used + kLazyRescale;
+        float alpha = 1.0f;
+        if (need) {
+          alpha = ptx::ex2(m_used - m_tile);
+          m_used = m_tile;
+        }
+        l *= alpha;
+        if (j > 0 && __any_sync(0xffffffffu, need)) scale_o(tO, alpha);
+        const uint64_t nm2 = ptx::f2_pack(-m_used, -m_used);
+        uint64_t acc[4] = {0, 0, 0, 0};
+        // reload 64 columns at a time; P of the first half overwrites S columns 0..31,
+        // already read, the second half's loads touch columns 64..127 only
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t sh[kBN / 2];
+          ptx::tmem_ld64(tS + 64 * hh, sh);
+          if (valid < kBN) {
+#pragma unroll
+            for (int i = 0; i < kBN / 2; ++i)
+              if (64 * hh + i >= valid) sh[i] = 0xff800000u;
+            softmax_half<false>(sh, c2, nm2, tS + 32 * hh, acc);
+          } else {
+            softmax_half<true>(sh, c2, nm2, tS + 32 * hh, acc);
+          }
+        }
+        float rs[4];
+        ptx::f2_unpack(ptx::f2_add(acc[0], acc[1]), rs[0], rs[1]);
+        ptx::f2_unpack(ptx::f2_add(acc[2], acc[3]), rs[2], rs[3]);
+        l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+      }
+      ptx::tmem_st_wait();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&bars[kBarPFull + wg]);
+    }
+    if (ok) {
+      ok = ptx::mbar_wait(&bars[kBarODone], 0, limit);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (!ok) {
+      if (lane == 0) atomicOr(p.status, kStatusTimeout);
+    } else {
+      ptx::tc_fence_after();
+      const int row = m0 + wg * kBM + r;
+      const bool live = row < p.Lq;
+      const float inv_l = 1.0f / l;
+      const long long base = (static_cast<long long>(row) * p.H + head) * kHeadDim;
+      FlowStep step;
+      step.sigma = p.sigma;
+      step.renoise = p.sigma_next >= 0.0;
+      step.sigma_next = step.renoise ? p.sigma_next : 0.0;
+      step.one_minus_next = __dsub_rn(1.0, step.sigma_next);
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t rr[32];
-          ptx::tmem_ld32(tO + 32 * c, rr);
-          if (live) {
-            uint32_t ob[16];
-            if (oth != nullptr) {
-              const float4* o4 = reinterpret_cast<const float4*>(oth + 32 * c);
+      for (int c = 0; c < 4; ++c) {
+        uint32_t rr[32];
+        ptx::tmem_ld32(tO + 32 * c, rr);
+        if (live) {
+          uint32_t ob[16];
 #pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const float4 w = __ldcg(o4 + i);
-                ob[2 * i] = pack_bf16x2(__uint_as_float(rr[4 * i]) * g_own + w.x * g_oth,
-                                        __uint_as_float(rr[4 * i + 1]) * g_own + w.y * g_oth);
-                ob[2 * i + 1] = pack_bf16x2(__uint_as_float(rr[4 * i + 2]) * g_own + w.z * g_oth,
-                                            __uint_as_float(rr[4 * i + 3]) * g_own + w.w * g_oth);
-              }
-            } else {
+          for (int i = 0; i < 16; ++i)
+            ob[i] = pack_bf16x2(__uint_as_float(rr[2 * i]) * inv_l, __uint_as_float(rr[2 * i + 1]) * inv_l);
+          uint4* dst = reinterpret_cast<uint4*>(p.out + base + 32 * c);
 #pragma unroll
-              for (int i = 0; i < 16; ++i)
-                ob[i] = pack_bf16x2(__uint_as_float(rr[2 * i]) * inv_l, __uint_as_float(rr[2 * i + 1]) * inv_l);
-            }
-            uint4* dst = reinterpret_cast<uint4*>(p.out + base + 32 * c);
+          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(ob[4 * v], ob[4 * v + 1], ob[4 * v + 2], ob[4 * v + 3]);
+          if (p.flow) {
+            const uint4* xtp = reinterpret_cast<const uint4*>(p.xt + base + 32 * c);
+            const uint4* ep = reinterpret_cast<const uint4*>(p.eps + base + 32 * c);
+            uint4* x0p = reinterpret_cast<uint4*>(p.x0 + base + 32 * c);
+            uint4* xnp = reinterpret_cast<uint4*>(p.xt_next + base + 32 * c);
+            const uint4* cp = reinterpret_cast<const uint4*>(p.v_cond + base + 32 * c);
+            const bool cfg = p.v_cond != nullptr;
 #pragma unroll
-            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(ob[4 * v], ob[4 * v + 1], ob[4 * v + 2], ob[4 * v + 3]);
-            if (p.flow) {
-              const uint4* xtp = reinterpret_cast<const uint4*>(p.xt + base + 32 * c);
-              const uint4* ep = reinterpret_cast<const uint4*>(p.eps + base + 32 * c);
-              uint4* x0p = reinterpret_cast<uint4*>(p.x0 + base + 32 * c);
-              uint4* xnp = reinterpret_cast<uint4*>(p.xt_next + base + 32 * c);
-              const uint4* cp = reinterpret_cast<const uint4*>(p.v_cond + base + 32 * c);
-              const bool cfg = p.v_cond != nullptr;
+            for (int v = 0; v < 4; ++v) {
+              const uint4 xv = __ldg(xtp + v);
+              uint4 ev = make_uint4(0, 0, 0, 0), cv = make_uint4(0, 0, 0, 0);
+              if (step.renoise) ev = __ldg(ep + v);
+              if (cfg) cv = __ldg(cp + v);
+              const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+              const uint32_t ew[4] = {ev.x, ev.y, ev.z, ev.w};
+              const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
+              uint32_t o0[4], o1[4];
 #pragma unroll
-              for (int v = 0; v < 4; ++v) {
-                const uint4 xv = __ldg(xtp + v);
-                uint4 ev = make_uint4(0, 0, 0, 0), cv = make_uint4(0, 0, 0, 0);
-                if (step.renoise) ev = __ldg(ep + v);
-                if (cfg) cv = __ldg(cp + v);
-                const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-                const uint32_t ew[4] = {ev.x, ev.y, ev.z, ev.w};
-                const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
-                uint32_t o0[4], o1[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                  const uint32_t vw = ob[4 * v + q];
-                  uint16_t a0, a1, b0 = 0, b1 = 0;
-                  if (cfg) {
-                    // this launch is the unconditional branch: its output is u
-                    step.apply_cfg_bits(xw[q], cw[q], vw, ew[q], p.cfg_scale, a0, b0);
-                    step.apply_cfg_bits(xw[q] >> 16, cw[q] >> 16, vw >> 16, ew[q] >> 16, p.cfg_scale, a1, b1);
-                  } else {
-                    step.apply_bits(xw[q], vw, ew[q], a0, b0);
-                    step.apply_bits(xw[q] >> 16, vw >> 16, ew[q] >> 16, a1, b1);
-                  }
-                  o0[q] = static_cast<uint32_t>(a0) | (static_cast<uint32_t>(a1) << 16);
-                  o1[q] = static_cast<uint32_t>(b0) | (static_cast<uint32_t>(b1) << 16);
+              for (int q = 0; q < 4; ++q) {
+                const uint32_t vw = ob[4 * v + q];
+                uint16_t a0, a1, b0 = 0, b1 = 0;
+                if (cfg) {
+                  // this launch is the unconditional branch: its output is u
+                  step.apply_cfg_bits(xw[q], cw[q], vw, ew[q], p.cfg_scale, a0, b0);
+                  step.apply_cfg_bits(xw[q] >> 16, cw[q] >> 16, vw >> 16, ew[q] >> 16, p.cfg_scale, a1, b1);
+                } else {
+                  step.apply_bits(xw[q], vw, ew[q], a0, b0);
+                  step.apply_bits(xw[q] >> 16, vw >> 16, ew[q] >> 16, a1, b1);
                 }
-                x0p[v] = make_uint4(o0[0], o0[1], o0[2], o0[3]);
-                if (step.renoise) xnp[v] = make_uint4(o1[0], o1[1], o1[2], o1[3]);
+                o0[q] = static_cast<uint32_t>(a0) | (static_cast<uint32_t>(a1) << 16);
+                o1[q] = static_cast<uint32_t>(b0) | (static_cast<uint32_t>(b1) << 16);
               }
+              x0p[v] = make_uint4(o0[0], o0[1], o0[2], o0[3]);
+              if (step.renoise) xnp[v] = make_uint4(o1[0], o1[1], o1[2], o1[3]);
             }
           }
         }
       }
     }
-    if (!ok && lane == 0) atomicOr(p.status, kStatusTimeout);
   }
 
   ptx::tc_fence_before();
@@ -693,8 +574,7 @@ cudaError_t launch_attention(const CUtensorMap& tm_q, const CUtensorMap& tm_k, c
     if (err != cudaSuccess) return err;
     configured_device = dev;
   }
-  const int units = (p.Lq + 2 * kBM - 1) / (2 * kBM) * p.H;
-  dim3 grid(p.sk_ctas > 0 ? p.sk_ctas : units);
+  dim3 grid((p.Lq + 2 * kBM - 1) / (2 * kBM), p.H);
   chunk_attention_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_q, tm_k, tm_vc, tm_vn, p);
   return cudaGetLastError();
 }

@@ -58,17 +58,12 @@ struct Layer {
   int n_text = 0;    // 0 = not set
   int text_cap = 0;  // tokens the buffers can hold
   CUtensorMap tm_tk, tm_tv;
-  // stream-K work split of the attention launch (allocated when a call can have more
-  // units than the device has SMs): partial results at the cut units, arrival counters
-  float* sk_part = nullptr;     // [n_sm][2][kSkPartFloats]
-  unsigned* sk_count = nullptr;  // [n_sm][8], even between launches
 };
 
 }  // namespace
 
 struct rkv_ctx {
   int layers = 0, H = 0, d = 0, T = 0, W = 0, S = 0, R = 0, mode = 0;
-  int n_sm = 0;  // multiprocessors of the device the handle was created on
   bool grid_set = false;
   int gh = 0, gw = 0, pt = 0, ph = 0, pw = 0;
   double theta = 0;
@@ -258,11 +253,7 @@ void free_layer(Layer& L) {
   cudaFree(L.qstage);
   cudaFree(L.text_k);
   cudaFree(L.text_v);
-  cudaFree(L.sk_part);
-  cudaFree(L.sk_count);
   L.k = L.v = L.rotk = L.qstage = L.text_k = L.text_v = nullptr;
-  L.sk_part = nullptr;
-  L.sk_count = nullptr;
   L.n_text = L.text_cap = 0;
 }
 
@@ -304,13 +295,6 @@ RKV_API int rkv_create(int layers, int H, int d, int tokens_per_frame, int windo
   int rc = RKV_OK;
   if (cudaMalloc(&h->status, sizeof(unsigned)) != cudaSuccess || cudaMemset(h->status, 0, sizeof(unsigned)) != cudaSuccess)
     rc = RKV_ERR_CUDA;
-  int dev = 0;
-  if (rc == RKV_OK && (cudaGetDevice(&dev) != cudaSuccess ||
-                       cudaDeviceGetAttribute(&h->n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess))
-    rc = RKV_ERR_CUDA;
-  // units of the largest call: blocks of 2 x 128 query rows per head
-  const long long max_units = (q_rows + 2 * rkv::kQueryBox - 1) / (2 * rkv::kQueryBox) * H;
-  const bool stream_k = max_units > h->n_sm;
   for (int l = 0; l < layers && rc == RKV_OK; ++l) {
     Layer& L = h->L[l];
     L.slot_frame.assign(window_frames, -1);
@@ -327,15 +311,6 @@ RKV_API int rkv_create(int layers, int H, int d, int tokens_per_frame, int windo
         cudaMemset(L.rotk, 0, rot_b) != cudaSuccess || cudaMemset(L.qstage, 0, q_b) != cudaSuccess) {
       rc = RKV_ERR_CUDA;
       break;
-    }
-    if (stream_k) {
-      const size_t part_b = static_cast<size_t>(h->n_sm) * 2 * rkv::kSkPartFloats * sizeof(float);
-      const size_t cnt_b = static_cast<size_t>(h->n_sm) * 8 * sizeof(unsigned);
-      if (cudaMalloc(&L.sk_part, part_b) != cudaSuccess || cudaMalloc(&L.sk_count, cnt_b) != cudaSuccess ||
-          cudaMemset(L.sk_count, 0, cnt_b) != cudaSuccess) {
-        rc = RKV_ERR_CUDA;
-        break;
-      }
     }
     if (!encode_head_major(&L.tm_q, L.qstage, static_cast<int>(q_rows), H, rkv::kQueryBox) ||
         !encode_head_major(&L.tm_k, L.rotk, static_cast<int>(rot_rows), H, rkv::kKeyBox) ||
@@ -561,14 +536,6 @@ int chunk_attention_impl(rkv_handle h, int layer, const void* q, const void* k, 
   }
   ap.status = h->status;
   ap.wait_limit_ns = h->wait_ns;
-  {
-    const int units = (ap.Lq + 2 * rkv::kQueryBox - 1) / (2 * rkv::kQueryBox) * ap.H;
-    if (L.sk_part != nullptr && units > h->n_sm && units % h->n_sm != 0) {
-      ap.sk_ctas = h->n_sm;
-      ap.sk_part = L.sk_part;
-      ap.sk_count = L.sk_count;
-    }
-  }
   CUtensorMap tm_vn;
   if (!encode_token_major(&tm_vn, v, C * T, h->H, rkv::kKeyBox)) return RKV_ERR_CUDA;
   const bool timed = h->timing && h->timing_n < h->timing_max;
@@ -817,9 +784,6 @@ RKV_API int rkv_reset(rkv_handle h) {
     if (cudaMemset(L.k, 0, ring_b) != cudaSuccess || cudaMemset(L.v, 0, ring_b) != cudaSuccess ||
         cudaMemset(L.rotk, 0, rot_b) != cudaSuccess)
       return RKV_ERR_CUDA;
-    if (L.sk_count != nullptr &&
-        cudaMemset(L.sk_count, 0, static_cast<size_t>(h->n_sm) * 8 * sizeof(unsigned)) != cudaSuccess)
-      return RKV_ERR_CUDA;
     L.committed = 0;
     std::fill(L.slot_frame.begin(), L.slot_frame.end(), -1);
     L.rot_f0 = -1;
@@ -897,16 +861,7 @@ RKV_API int rkv_poll_device_status(rkv_handle h, void* stream) {
   unsigned word = 0;
   if (cudaMemcpy(&word, h->status, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return RKV_ERR_CUDA;
   if (word != 0 && cudaMemset(h->status, 0, sizeof(unsigned)) != cudaSuccess) return RKV_ERR_CUDA;
-  if (word & rkv::kStatusTimeout) {
-    // a launch that gave up may have left a stream-K arrival counter odd
-    if (cudaDeviceSynchronize() != cudaSuccess) return RKV_ERR_CUDA;
-    for (Layer& L : h->L)
-      if (L.sk_count != nullptr &&
-          cudaMemset(L.sk_count, 0, static_cast<size_t>(h->n_sm) * 8 * sizeof(unsigned)) != cudaSuccess)
-        return RKV_ERR_CUDA;
-    return RKV_ERR_TIMEOUT;
-  }
-  return RKV_OK;
+  return (word & rkv::kStatusTimeout) ? RKV_ERR_TIMEOUT : RKV_OK;
 }
 
 RKV_API int rkv_set_wait_limit(rkv_handle h, long long nanoseconds) {

@@ -97,20 +97,7 @@ struct AttnParams {
   double cfg_scale;
   unsigned* status;
   unsigned long long wait_limit_ns;
-  // Work split. A unit is one head x one block of 2 * kQueryBox query rows against the whole
-  // key stream (n_tiles key tiles). sk_ctas == 0: one CTA per unit. sk_ctas > 0: a persistent
-  // launch of sk_ctas CTAs, CTA c taking the tiles [c T / sk_ctas, (c + 1) T / sk_ctas) of the
-  // T = units x n_tiles (unit, tile) pairs in order ("stream-K"), which needs units > sk_ctas;
-  // a unit cut by boundary b is finished by whichever of its two CTAs arrives second
-  // (sk_count[b] parity), from the other's partial result in sk_part.
-  int sk_ctas;
-  float* sk_part;      // [sk_ctas][2][kSkPartFloats]
-  unsigned* sk_count;  // [sk_ctas], even between launches
 };
-
-// Floats of one partial result: O (unnormalised) [2 * kQueryBox][kHeadDim], then the
-// reference m and the sum l of each row.
-constexpr int kSkPartFloats = 2 * kQueryBox * (kHeadDim + 2);
 
 cudaError_t launch_attention(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_vc,
                              const CUtensorMap& tm_vn, const AttnParams& p, cudaStream_t stream);
