@@ -28,6 +28,8 @@ FULL = [
     (Config("480p", 21, H=40, grid_h=30, grid_w=52, C=4, W=18, S=6, rope_mode=ABS, chunks=6, reads=1), (1, 4, 5)),
     # the ABot shape with slot-order relative ids (the five reference sinks keep ids 0..4)
     (Config("abot-slots", 23, H=24, grid_h=22, grid_w=40, C=3, W=21, S=5, rope_mode=SLOTS, refs=5, chunks=7, reads=1), (6,)),
+    # 16 heads x 10 query blocks = 160 CTAs, more than the 148 SMs: a second, partial wave
+    (Config("many-units", 24, H=16, grid_h=32, grid_w=40, C=2, W=5, S=1, rope_mode=ABS, chunks=5, reads=1), (1, 2, 4)),
     (Config("720p", 22, H=40, grid_h=45, grid_w=80, C=4, W=18, S=6, rope_mode=ABS, chunks=5, reads=1), (4,)),
 ]
 
