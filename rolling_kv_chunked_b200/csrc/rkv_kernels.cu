@@ -125,7 +125,9 @@ __device__ __forceinline__ uint4 flow_x0(const FlowStep& step, double scale, uin
   return make_uint4(ow[0], ow[1], ow[2], ow[3]);
 }
 
-// Two 16-byte vectors per thread per iteration, all loads issued before the arithmetic.
+// One 16-byte vector of each operand per thread per iteration. The bf16 <-> fp64
+// conversions run on the special-function unit and keep it busy, so HBM stays busy only
+// with many resident warps: few registers per thread (40) and a grid of 16 blocks per SM.
 template <bool kCfg>
 __global__ void __launch_bounds__(256) flow_kernel(const FlowParams p) {
   FlowStep step;
@@ -142,27 +144,14 @@ __global__ void __launch_bounds__(256) flow_kernel(const FlowParams p) {
   const uint4* ep = reinterpret_cast<const uint4*>(p.eps);
   uint4* x0p = reinterpret_cast<uint4*>(p.x0);
   uint4* xnp = reinterpret_cast<uint4*>(p.xt_next);
-  for (long long i = gid; i < n_vec; i += 2 * threads) {
-    const long long i2 = i + threads;
-    const bool two = i2 < n_vec;
+  for (long long i = gid; i < n_vec; i += threads) {
     const uint4 zero = make_uint4(0, 0, 0, 0);
     const uint4 xa = __ldg(xtp + i), va = __ldg(vp + i);
     const uint4 ua = kCfg ? __ldg(up + i) : zero;
     const uint4 ea = step.renoise ? __ldg(ep + i) : zero;
-    uint4 xb = zero, vb = zero, ub = zero, eb = zero;
-    if (two) {
-      xb = __ldg(xtp + i2);
-      vb = __ldg(vp + i2);
-      if (kCfg) ub = __ldg(up + i2);
-      if (step.renoise) eb = __ldg(ep + i2);
-    }
-    uint4 na, nb;
+    uint4 na;
     x0p[i] = flow_x0<kCfg>(step, p.cfg_scale, xa, va, ua, ea, na);
     if (step.renoise) xnp[i] = na;
-    if (two) {
-      x0p[i2] = flow_x0<kCfg>(step, p.cfg_scale, xb, vb, ub, eb, nb);
-      if (step.renoise) xnp[i2] = nb;
-    }
   }
   // ragged tail (n not a multiple of 8): one element per thread of the first block
   const long long tail0 = n_vec << 3;
@@ -196,7 +185,7 @@ cudaError_t launch_flow(const FlowParams& p, cudaStream_t stream) {
   if (p.n <= 0) return cudaSuccess;
   const long long vecs = std::max(1LL, p.n >> 3);
   long long blocks = (vecs + 255) / 256;
-  const long long cap = static_cast<long long>(sm_count()) * 8;
+  const long long cap = static_cast<long long>(sm_count()) * 16;
   blocks = std::max(1LL, std::min(blocks, cap));
   if (p.v_uncond != nullptr) {
     flow_kernel<true><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
