@@ -304,6 +304,27 @@ int rkv_timing_end(rkv_handle h, float* ms_out, int max, int* n_out);
 int rkv_plan_window(int window_frames, int sink_frames, int frames_committed, int n_frames,
                     int start_frame, int* seg_out, int max_segs, int* n_segs);
 
+/*
+ * rkv_copy_heads - strided copies of per-head vectors (d = 128 bf16 each), the data
+ *  movement around the sequence <-> head exchange of head-sharded attention
+ *  ("从40步到4步..." / LingBot-World `wan/` source map, §多卡加速: Ulysses sequence
+ *  parallelism, an all-to-all before and after attention with ulysses_size | num_heads).
+ *  Each of the n_runs records copies n_tok tokens x n_heads heads: head vector (t, h)
+ *  moves from src + t * src_tok_stride + h * src_head_stride to the same offsets in dst
+ *  (strides in bf16 elements, multiples of 8; src and dst 16-byte aligned, not
+ *  overlapping). Device pointers; asynchronous on `stream`; runs are issued up to eight
+ *  per kernel launch. A bit copy: no arithmetic. Errors: RKV_ERR_ARG (null or misaligned
+ *  pointer, negative count or stride not a multiple of 8, n_heads < 1), RKV_ERR_CUDA.
+ */
+typedef struct rkv_head_copy {
+  const void* src;
+  void* dst;
+  long long src_tok_stride, src_head_stride;
+  long long dst_tok_stride, dst_head_stride;
+  int n_tok;
+} rkv_head_copy;
+int rkv_copy_heads(const rkv_head_copy* runs, int n_runs, int n_heads, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

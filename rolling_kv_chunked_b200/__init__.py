@@ -44,6 +44,12 @@ class FlowEpilogue(ctypes.Structure):
                 ("x0_out", _vp), ("xt_next_out", _vp)]
 
 
+class HeadCopy(ctypes.Structure):
+    """Mirror of ``rkv_head_copy``: n_tok tokens x n_heads head vectors, strides in elements."""
+    _fields_ = [("src", _vp), ("dst", _vp), ("src_tok_stride", _c_ll), ("src_head_stride", _c_ll),
+                ("dst_tok_stride", _c_ll), ("dst_head_stride", _c_ll), ("n_tok", _c_int)]
+
+
 _SIGS = {
     "rkv_create": ([_c_int] * 7 + [ctypes.POINTER(_vp)], _c_int),
     "rkv_set_rope_grid": ([_vp, _c_int, _c_int, _c_dbl, _c_int, _c_int, _c_int], _c_int),
@@ -70,6 +76,7 @@ _SIGS = {
     "rkv_timing_begin": ([_vp, _c_int], _c_int),
     "rkv_timing_end": ([_vp, ctypes.POINTER(ctypes.c_float), _c_int, _int_p], _c_int),
     "rkv_plan_window": ([_c_int, _c_int, _c_int, _c_int, _c_int, _int_p, _c_int, _int_p], _c_int),
+    "rkv_copy_heads": ([ctypes.POINTER(HeadCopy), _c_int, _c_int, _vp], _c_int),
 }
 for _name, (_args, _res) in _SIGS.items():
     try:
@@ -129,6 +136,15 @@ def flow_x0_renoise(xt, v, eps, sigma: float, sigma_next: float, x0_out, xt_next
     _check(_lib.rkv_flow_x0_renoise(_ptr(xt), _ptr(v), _ptr(eps), float(sigma), float(sigma_next),
                                     _ptr(x0_out), _ptr(xt_next_out), xt.numel(), _stream(stream)),
            "rkv_flow_x0_renoise")
+
+
+def copy_heads(runs, n_heads: int, stream=None) -> None:
+    """Strided head-vector copies. ``runs``: (src_ptr, dst_ptr, src_tok_stride, src_head_stride,
+    dst_tok_stride, dst_head_stride, n_tok) tuples, pointers as ints, strides in elements."""
+    arr = (HeadCopy * max(1, len(runs)))()
+    for i, r in enumerate(runs):
+        arr[i] = HeadCopy(*r)
+    _check(_lib.rkv_copy_heads(arr, len(runs), int(n_heads), _stream(stream)), "rkv_copy_heads")
 
 
 def flow_cfg_x0_renoise(xt, v_cond, v_uncond, eps, cfg_scale: float, sigma: float, sigma_next: float, x0_out,

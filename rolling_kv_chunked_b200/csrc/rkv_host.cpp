@@ -708,6 +708,44 @@ RKV_API int rkv_rope_apply(rkv_handle h, void* x, int n_frames, int start_frame,
   return cuda_rc(rkv::launch_frame_runs(p, max_tok, static_cast<cudaStream_t>(stream)));
 }
 
+RKV_API int rkv_copy_heads(const rkv_head_copy* runs, int n_runs, int n_heads, void* stream) {
+  if (n_runs < 0 || (n_runs > 0 && runs == nullptr) || n_heads < 1) return RKV_ERR_ARG;
+  for (int i = 0; i < n_runs; ++i) {
+    const rkv_head_copy& c = runs[i];
+    if (c.n_tok < 0 || !aligned16(c.src) || !aligned16(c.dst)) return RKV_ERR_ARG;
+    if (c.n_tok > 0 && (c.src == nullptr || c.dst == nullptr)) return RKV_ERR_ARG;
+    for (long long st : {c.src_tok_stride, c.src_head_stride, c.dst_tok_stride, c.dst_head_stride})
+      if (st < 0 || st % 8 != 0) return RKV_ERR_ARG;
+  }
+  for (int i0 = 0; i0 < n_runs; i0 += rkv::kMaxRuns) {
+    FrameRunParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.H = n_heads;
+    p.T = 1;
+    p.grid_w = 1;
+    int max_tok = 0;
+    for (int i = i0; i < n_runs && i < i0 + rkv::kMaxRuns; ++i) {
+      const rkv_head_copy& c = runs[i];
+      if (c.n_tok == 0) continue;
+      FrameRun r;
+      std::memset(&r, 0, sizeof(r));
+      r.src = static_cast<const uint16_t*>(c.src);
+      r.dst = static_cast<uint16_t*>(c.dst);
+      r.src_tok_stride = c.src_tok_stride;
+      r.src_head_stride = c.src_head_stride;
+      r.dst_tok_stride = c.dst_tok_stride;
+      r.dst_head_stride = c.dst_head_stride;
+      r.n_tok = c.n_tok;
+      r.rotate = 0;
+      add_run(p, r);
+      max_tok = std::max(max_tok, c.n_tok);
+    }
+    const int rc = cuda_rc(rkv::launch_frame_runs(p, max_tok, static_cast<cudaStream_t>(stream)));
+    if (rc) return rc;
+  }
+  return RKV_OK;
+}
+
 RKV_API int rkv_flow_x0_renoise(const void* xt, const void* v, const void* eps, double sigma, double sigma_next,
                                 void* x0_out, void* xt_next_out, long long n, void* stream) {
   if (n < 0) return RKV_ERR_ARG;

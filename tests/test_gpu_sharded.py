@@ -1,0 +1,145 @@
+"""Head-sharded attention on the GPU kernels: two ranks emulated in one process on one GPU.
+
+Each emulated rank is a HeadShardedRollingKV (its own caches of H/2 heads); the phases run
+with this library's kernels (rkv_copy_heads packs / unpacks the head blocks, the chunk
+attention runs per rank) and the all-to-all between the ranks is done in-process by the
+test (copies of the ranks' send slices; no collective, nothing waits on another rank).
+Checked against one unsharded RollingKV of all heads on the same inputs: every output
+block bit for bit, through sinks, warm-up, eviction and wrap, both RoPE modes, and the x0 /
+renoise step on each rank's latent block bit for bit against the unsharded fused epilogue;
+the caches of each rank equal the unsharded cache's heads bit for bit; rkv_copy_heads
+against numpy slicing and its argument errors.
+"""
+import numpy as np
+import pytest
+
+import synth
+from rollout import to_bits
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("no CUDA device", allow_module_level=True)
+
+import rolling_kv_chunked_b200 as rkv  # noqa: E402
+from rolling_kv_chunked_b200.sharded import HeadShardedRollingKV  # noqa: E402
+
+H, GH, GW, C, W, S, G = 4, 8, 10, 2, 6, 2, 2
+T = GH * GW
+
+
+def _dev(key, shape):
+    t = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+    synth.fill_normal_bf16_cuda(t.data_ptr(), t.numel(), key, 0, torch.cuda.current_stream().cuda_stream)
+    return t
+
+
+def _exchange(sends):
+    """All-to-all among the emulated ranks: rank j receives slice j of every rank's send."""
+    return [torch.stack([sends[i][j] for i in range(G)]) for j in range(G)]
+
+
+def _sharded_call(ranks, *tensors, n_frames):
+    """Pack each rank's token blocks, exchange, and return every rank's [Lq, H/G, d] inputs."""
+    per_rank = []
+    for x in tensors:
+        sends = [ranks[r].pack(x[r], n_frames) for r in range(G)]
+        per_rank.append([t.view(-1, H // G, 128) for t in _exchange(sends)])
+    return per_rank
+
+
+@pytest.mark.parametrize("mode", [rkv.ROPE_ABSOLUTE, rkv.ROPE_RELATIVE])
+def test_two_emulated_ranks_match_unsharded_bit_for_bit(mode):
+    ranks = [HeadShardedRollingKV(1, H, 128, T, W, S, mode, world_size=G, rank=r) for r in range(G)]
+    full = rkv.RollingKV(1, H, 128, T, W, S, mode)
+    for h in ranks + [full]:
+        h.set_rope_grid(GH, GW)
+    Lq = C * T
+    Lb = Lq // G
+
+    def blocks(x, n_tok):
+        b = n_tok // G
+        return [x[r * b:(r + 1) * b].contiguous() for r in range(G)]
+
+    # sinks written without attention
+    kr, vr = _dev(synth.stream_key(6, 1), (S * T, H, 128)), _dev(synth.stream_key(6, 2), (S * T, H, 128))
+    (k_in, v_in) = _sharded_call(ranks, blocks(kr, S * T), blocks(vr, S * T), n_frames=S)
+    for r in range(G):
+        ranks[r].local.write_chunk(0, k_in[r], v_in[r], S, 0)
+    full.write_chunk(0, kr, vr, S, 0)
+    f0 = S
+    sig = [1.0, 0.75]
+    for chunk in range(5):
+        xt = _dev(synth.stream_key(6, 3, chunk), (Lq, H * 128))
+        for call in range(2):
+            commit = call == 1
+            q, k, v = (_dev(synth.stream_key(6, 4, chunk, call, t), (Lq, H, 128)) for t in range(3))
+            eps = _dev(synth.stream_key(6, 5, chunk, call), (Lq, H * 128))
+            out_full = torch.empty((Lq, H, 128), dtype=torch.bfloat16, device="cuda")
+            x0_full, xn_full = torch.empty_like(xt), torch.empty_like(xt)
+            if commit:
+                full.chunk_attention(0, q, k, v, out_full, C, f0, True)
+            else:
+                full.chunk_attention(0, q, k, v, out_full, C, f0, False,
+                                     flow=dict(xt=xt, eps=eps, sigma=sig[0], sigma_next=sig[1],
+                                               x0_out=x0_full, xt_next_out=xn_full))
+            qs, ks, vs = _sharded_call(ranks, blocks(q, Lq), blocks(k, Lq), blocks(v, Lq), n_frames=C)
+            outs_h = [ranks[r].attend(0, qs[r], ks[r], vs[r], C, f0, commit) for r in range(G)]
+            back = _exchange([o.view(G, Lb, H // G, 128) for o in outs_h])
+            for r in range(G):
+                out_r = torch.empty((Lb, H, 128), dtype=torch.bfloat16, device="cuda")
+                ranks[r].unpack(back[r], out_r, C)
+                torch.cuda.synchronize()
+                assert np.array_equal(to_bits(out_r), to_bits(out_full[r * Lb:(r + 1) * Lb])), (mode, chunk, call, r)
+                if not commit:
+                    xb = xt[r * Lb:(r + 1) * Lb].contiguous()
+                    eb = eps[r * Lb:(r + 1) * Lb].contiguous()
+                    x0_r, xn_r = torch.empty_like(xb), torch.empty_like(xb)
+                    rkv.flow_x0_renoise(xb, out_r.view(Lb, H * 128), eb, sig[0], sig[1], x0_r, xn_r)
+                    torch.cuda.synchronize()
+                    assert np.array_equal(to_bits(x0_r), to_bits(x0_full[r * Lb:(r + 1) * Lb]))
+                    assert np.array_equal(to_bits(xn_r), to_bits(xn_full[r * Lb:(r + 1) * Lb]))
+        f0 += C
+    # each rank's cache holds exactly the unsharded cache's heads
+    n_el = W * T * 128
+    for which in range(2):
+        fp = full.cache_ptrs(0)[which]
+        full_c = torch.as_tensor(_Arr(fp, H * n_el), device="cuda").view(torch.bfloat16).view(H, W * T, 128)
+        for r in range(G):
+            rp = ranks[r].local.cache_ptrs(0)[which]
+            rc = torch.as_tensor(_Arr(rp, (H // G) * n_el), device="cuda").view(torch.bfloat16).view(H // G, W * T, 128)
+            assert np.array_equal(to_bits(rc), to_bits(full_c[r * (H // G):(r + 1) * (H // G)]))
+        assert ranks[0].local.slot_frames(0) == full.slot_frames(0) == ranks[1].local.slot_frames(0)
+    for h in ranks:
+        h.close()
+    full.close()
+
+
+class _Arr:
+    def __init__(self, ptr, n):
+        self.__cuda_array_interface__ = {"shape": (n,), "typestr": "<i2", "data": (ptr, False), "version": 3}
+
+
+def test_copy_heads_strided_blocks_and_errors():
+    n_tok, Hs, Hd = 37, 6, 3   # 3 of 6 heads, ragged token count
+    x = _dev(synth.stream_key(6, 9), (n_tok, Hs, 128))
+    y = torch.zeros((2, n_tok, Hd, 128), dtype=torch.bfloat16, device="cuda")
+    runs = [(x.data_ptr() + r * Hd * 128 * 2, y[r].data_ptr(), Hs * 128, 128, Hd * 128, 128, n_tok) for r in range(2)]
+    rkv.copy_heads(runs, Hd)
+    torch.cuda.synchronize()
+    xb = to_bits(x)
+    for r in range(2):
+        assert np.array_equal(to_bits(y[r]), xb[:, r * Hd:(r + 1) * Hd, :])
+    # more runs than one launch takes (nine), zero-token runs skipped
+    many = [(x.data_ptr(), y[0].data_ptr(), Hs * 128, 128, Hd * 128, 128, n_tok if i % 3 else 0) for i in range(9)]
+    rkv.copy_heads(many, Hd)
+    torch.cuda.synchronize()
+    assert np.array_equal(to_bits(y[0]), xb[:, :Hd, :])
+    for bad in [(x.data_ptr() + 2, y[0].data_ptr(), Hs * 128, 128, Hd * 128, 128, 4),   # misaligned
+                (x.data_ptr(), y[0].data_ptr(), Hs * 128 + 4, 128, Hd * 128, 128, 4),   # stride not a multiple of 8
+                (x.data_ptr(), y[0].data_ptr(), Hs * 128, 128, Hd * 128, 128, -1)]:     # negative count
+        with pytest.raises(rkv.RkvError):
+            rkv.copy_heads([bad], Hd)
+    with pytest.raises(rkv.RkvError):
+        rkv.copy_heads(runs, 0)
