@@ -102,13 +102,14 @@ def peaks():
 
 # ---------------------------------------------------------------------- clocks
 class ClockSampler:
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_id: str | None):
         self.proc = None
         self.path = None
+        self.window = [None, None]
         if gpu_id is None:
             return
         try:
@@ -121,7 +122,18 @@ class ClockSampler:
         except (OSError, FileNotFoundError):
             self.proc = None
 
+    def mark_start(self):
+        import datetime
+        self.window[0] = datetime.datetime.now()
+
+    def mark_end(self):
+        import datetime
+        self.window[1] = datetime.datetime.now()
+
     def stop(self):
+        """Median SM clock and throttle reasons of the samples taken inside the marked window
+        (all samples if none fell inside it)."""
+        import datetime
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -130,28 +142,32 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.fh.close()
-        sm, mx, reasons = [], None, set()
+        rows, mx = [], None
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         with open(self.path) as fh:
             for line in fh:
                 parts = [x.strip() for x in line.split(",")]
-                if len(parts) < 8:
+                if len(parts) < 9:
                     continue
                 try:
-                    sm.append(float(parts[0]))
-                    mx = float(parts[1])
+                    ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f")
+                    rows.append((ts, float(parts[1]), [n for n, v in zip(names, parts[5:9]) if v.lower() == "active"]))
+                    mx = float(parts[2])
                 except ValueError:
                     continue
-                for n, val in zip(names, parts[4:8]):
-                    if val.lower() == "active":
-                        reasons.add(n)
+        t0, t1 = self.window
+        inside = [r for r in rows if t0 is not None and t1 is not None and t0 <= r[0] <= t1]
+        use = inside if inside else rows
+        sm = [r[1] for r in use]
+        reasons = {n for r in use for n in r[2]}
         try:
             os.remove(self.path)
         except OSError:
             pass
         if not sm:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm),
+                "samples_in_timed_region": len(inside)}
 
 
 # ---------------------------------------------------------------------- ranks
@@ -252,6 +268,12 @@ def run_rkv(args):
         inp = pool[i % pool_n]
         h.chunk_attention(0, inp["q"][4], inp["k"][4], inp["v"][4], outs[4], C, state["f0"], True, stream=sp)
         state["f0"] += C
+    gpu_id = None
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
+    except Exception:
+        gpu_id = None
+    clocks = ClockSampler(gpu_id)  # started before the warm-up, so that it samples from the first timed step
     for i in range(args.warmup):
         step(pool[i % pool_n])
     torch.cuda.synchronize()
@@ -265,15 +287,10 @@ def run_rkv(args):
         flops += 5 * 4.0 * H * 128 * Lq * visible_keys(cfg, f, f)
         f += C
 
-    gpu_id = None
-    try:
-        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
-    except Exception:
-        gpu_id = None
-    clocks = ClockSampler(gpu_id)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    clocks.mark_start()
     h.timing_begin(5 * args.steps)
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
@@ -282,6 +299,7 @@ def run_rkv(args):
         step(pool[i % pool_n])
     ev1.record(stream)
     torch.cuda.synchronize()
+    clocks.mark_end()
     kernel_ms = h.timing_end(5 * args.steps)
     if world > 1:
         dist.barrier()
@@ -402,6 +420,12 @@ def run_cfg(args):
         for br in range(2):
             hs[br].chunk_attention(0, *qkv[br][n_sets - 1], outs[br], C, state["f0"], True, stream=sp)
         state["f0"] += C
+    gpu_id = None
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
+    except Exception:
+        gpu_id = None
+    clocks = ClockSampler(gpu_id)  # started before the warm-up, so that it samples from the first timed step
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -410,13 +434,8 @@ def run_cfg(args):
     for _ in range(args.steps):
         flops += calls * 4.0 * H * 128 * Lq * visible_keys(cfg, f, f)
         f += C
-    gpu_id = None
-    try:
-        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
-    except Exception:
-        gpu_id = None
-    clocks = ClockSampler(gpu_id)
     torch.cuda.synchronize()
+    clocks.mark_start()
     for h in hs:
         h.timing_begin(calls * args.steps)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -425,6 +444,7 @@ def run_cfg(args):
         step()
     ev1.record(stream)
     torch.cuda.synchronize()
+    clocks.mark_end()
     kernel_ms = hs[0].timing_end(calls * args.steps) + hs[1].timing_end(calls * args.steps)
     clk = clocks.stop()
     ms = ev0.elapsed_time(ev1)
@@ -564,28 +584,42 @@ def measure_hbm_kernels(torch, rkv, synth, cfg, rank, reps=20):
         return t
 
     def timed(fn):
+        """Seconds per launch: `reps` launches captured in one CUDA graph and replayed, so that
+        the host's per-call overhead does not leave the GPU idle between small launches (the
+        launches, their arguments and their buffers are the same as when called directly)."""
         fn(0)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        graph = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream()
+        cap.wait_stream(st)
+        with torch.cuda.stream(cap):
+            graph.capture_begin()
+            for i in range(reps):
+                fn(i, cap.cuda_stream)
+            graph.capture_end()
+        st.wait_stream(cap)
+        graph.replay()
+        torch.cuda.synchronize()
         e0.record(st)
-        for i in range(reps):
-            fn(i)
+        graph.replay()
         e1.record(st)
         torch.cuda.synchronize()
+        del graph
         return e0.elapsed_time(e1) / reps / 1e3
 
     res = {}
     # K4: x0 = xt - sigma v; xt' = (1 - sigma') x0 + sigma' eps; 3 reads + 2 writes of bf16
     sets = [[fill(torch.empty(n, **bf), i, j) for j in range(5)] for i in range(n_sets)]
-    sec = timed(lambda i: rkv.flow_x0_renoise(sets[i % n_sets][0], sets[i % n_sets][1], sets[i % n_sets][2],
-                                              1.0, 0.75, sets[i % n_sets][3], sets[i % n_sets][4], stream=sp))
+    sec = timed(lambda i, s=sp: rkv.flow_x0_renoise(sets[i % n_sets][0], sets[i % n_sets][1], sets[i % n_sets][2],
+                                                    1.0, 0.75, sets[i % n_sets][3], sets[i % n_sets][4], stream=s))
     res["flow_x0_renoise"] = {"bytes_per_launch": 10 * n, "GB/s": 10 * n / sec / 1e9}
     del sets
     # K3: in-place RoPE of a [Lq, H, 128] tensor, one read + one write
     bufs = [fill(torch.empty((Lq, H, 128), **bf), 50, i) for i in range(2 * n_sets)]
     hr = rkv.RollingKV(1, H, 128, T, W, S, cfg["mode"])
     hr.set_rope_grid(cfg["gh"], cfg["gw"])
-    sec = timed(lambda i: hr.rope_apply(bufs[i % len(bufs)], C, 0, C, stream=sp))
+    sec = timed(lambda i, s=sp: hr.rope_apply(bufs[i % len(bufs)], C, 0, C, stream=s))
     res["rope_apply"] = {"bytes_per_launch": 4 * n, "GB/s": 4 * n / sec / 1e9}
     # K1: the ring write-back (rkv_write_chunk): K and V read and written once; in absolute
     # mode the rotated copy of K is written as well
@@ -593,8 +627,8 @@ def measure_hbm_kernels(torch, rkv, synth, cfg, rank, reps=20):
     hw.set_rope_grid(cfg["gh"], cfg["gw"])
     state = {"f": 0}
 
-    def write(i):
-        hw.write_chunk(0, bufs[(2 * i) % len(bufs)], bufs[(2 * i + 1) % len(bufs)], C, state["f"], stream=sp)
+    def write(i, s=sp):
+        hw.write_chunk(0, bufs[(2 * i) % len(bufs)], bufs[(2 * i + 1) % len(bufs)], C, state["f"], stream=s)
         state["f"] += C
     sec = timed(write)
     per = 8 * n + (4 * n if cfg["mode"] == 0 else 0)
