@@ -58,9 +58,9 @@ __device__ __forceinline__ uint4 rotate_vec(uint4 val, const float2 (&cs)[4]) {
 }
 
 // One warp per token. Lane l always handles the 16-byte vector l % 16 of heads
-// l / 16, l / 16 + 2, ... (four heads in flight), so a half-warp moves one head's 256
-// contiguous bytes per instruction and each lane fetches its four (cos, sin) pairs once per
-// token. blockIdx.y selects the run.
+// l / 16, l / 16 + 2, ... (eight heads in flight, their loads issued before the (cos, sin)
+// lookups), so a half-warp moves one head's 256 contiguous bytes per instruction and each
+// lane fetches its four (cos, sin) pairs once per eight heads. blockIdx.y selects the run.
 __global__ void __launch_bounds__(256) frame_runs_kernel(const __grid_constant__ FrameRunParams p) {
   const int r = blockIdx.y;
   if (r >= p.n_runs) return;
@@ -72,22 +72,22 @@ __global__ void __launch_bounds__(256) frame_runs_kernel(const __grid_constant__
   for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < run.n_tok; t += warps) {
     const uint16_t* src = run.src + static_cast<long long>(run.src_tok0 + t) * run.src_tok_stride + vec * 8;
     uint16_t* dst = run.dst + static_cast<long long>(run.dst_tok0 + t) * run.dst_tok_stride + vec * 8;
-    float2 cs[4];
-    if (run.rotate) {
-      const int frame = t / p.T;
-      const int tok = t - frame * p.T;
-      const int hh = tok / p.grid_w;
-      pair_cos_sin(vec, min(max(run.t0 + frame, p.t_lo), p.t_hi), hh, tok - hh * p.grid_w, p, cs);
-    }
-    for (int hb = h0; hb < p.H; hb += 8) {
-      uint4 val[4];
+    for (int hb = h0; hb < p.H; hb += 2 * 8) {
+      uint4 val[8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 8; ++u) {
         const int h = hb + 2 * u;
         if (h < p.H) val[u] = __ldg(reinterpret_cast<const uint4*>(src + h * run.src_head_stride));
       }
+      float2 cs[4];
+      if (run.rotate) {
+        const int frame = t / p.T;
+        const int tok = t - frame * p.T;
+        const int hh = tok / p.grid_w;
+        pair_cos_sin(vec, min(max(run.t0 + frame, p.t_lo), p.t_hi), hh, tok - hh * p.grid_w, p, cs);
+      }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 8; ++u) {
         const int h = hb + 2 * u;
         if (h < p.H) {
           uint4 v = val[u];
