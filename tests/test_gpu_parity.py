@@ -193,6 +193,43 @@ def test_score_jumps_between_key_tiles(sink_score, mode):
     h.close()
 
 
+@pytest.mark.parametrize("mode", [REL, SLOTS, ABS])
+def test_relative_translation_invariance_bitwise(mode):
+    """Identical raw window contents at two chunks whose ring layout is the same (chunks 6 and
+    6 + R, contents repeating every R chunks) give bit-identical GPU outputs in both relative
+    modes (the ids depend only on a frame's place in the window); absolute ids make them differ."""
+    H, gh, gw, C, W, S = 2, 8, 10, 2, 6, 2
+    T = gh * gw
+    R = W - S
+    h = rkv.RollingKV(1, H, 128, T, W, S, mode)
+    h.set_rope_grid(gh, gw)
+    stream = torch.cuda.current_stream().cuda_stream
+
+    def fill(*key):
+        t = torch.empty((C * T, H, 128), dtype=torch.bfloat16, device="cuda")
+        synth.fill_normal_bf16_cuda(t.data_ptr(), t.numel(), synth.stream_key(8, *key), 0, stream)
+        return t
+
+    sink_k = torch.empty((S * T, H, 128), dtype=torch.bfloat16, device="cuda")
+    sink_v = torch.empty_like(sink_k)
+    synth.fill_normal_bf16_cuda(sink_k.data_ptr(), sink_k.numel(), synth.stream_key(8, 99, 1), 0, stream)
+    synth.fill_normal_bf16_cuda(sink_v.data_ptr(), sink_v.numel(), synth.stream_key(8, 99, 2), 0, stream)
+    h.write_chunk(0, sink_k, sink_v, S, 0)
+    outs = {}
+    f0 = S
+    for c in range(6 + R + 1):
+        key = c % R
+        out = torch.empty((C * T, H, 128), dtype=torch.bfloat16, device="cuda")
+        h.chunk_attention(0, fill(key, 0), fill(key, 1), fill(key, 2), out, C, f0, False)
+        outs[c] = to_bits(out)
+        h.chunk_attention(0, fill(key, 3), fill(key, 4), fill(key, 5), out, C, f0, True)
+        f0 += C
+    torch.cuda.synchronize()
+    same = np.array_equal(outs[6], outs[6 + R])
+    assert same == (mode != ABS), mode
+    h.close()
+
+
 def test_host_errors_launch_nothing():
     cfg = Config("err", 10, H=2, grid_h=4, grid_w=4, C=2, W=6, S=2, rope_mode=ABS)
     h = rkv.RollingKV(1, cfg.H, 128, cfg.T, cfg.W, cfg.S, cfg.rope_mode)
