@@ -9,13 +9,15 @@ RoPE (relative or absolute) runs on the way in. Inputs are synthetic (seeded
 counter-based generator), resident in HBM before timing; the cache is rolled
 to steady state (full window, evictions firing) before warm-up.
 
-Metric: query tokens / s per layer (5 * Lq per step), whole job over all ranks.
+Metric: query tokens / s per layer (5 * Lq per layer per step), whole job over all ranks.
 Multi-GPU: independent replicas (one layer each), no data-path collective.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config abot|480p|720p|abot_cfg] [--impl rkv|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config abot|480p|720p|long|abot_cfg] [--impl rkv|reference]
 
 ``--config abot_cfg`` measures the guided (classifier-free guidance) mode instead: two caches,
 40 guided steps per chunk with the guidance combine fused into the unconditional read.
+``--config long`` stacks the ABot layer 30 deep (one cache per layer): each step is one chunk
+through all 30 layers.
 """
 from __future__ import annotations
 
@@ -49,6 +51,13 @@ CONFIGS = {
                           "[14400 x 5120] latent, 4 denoise reads + 1 commit per chunk",
                  H=40, gh=45, gw=80, C=4, W=18, S=6, refs=0, mode=0),
 }
+# the long-rollout stress shape: the ABot layer stacked 30 deep, one rolling cache per layer,
+# every step = one chunk through all layers (the layers reuse one seeded input set per call;
+# the caches, 6.8 GB in all, are per layer)
+CONFIGS["long"] = dict(CONFIGS["abot"], layers=30, workload=(
+    "Long rollout stress: ABot shape (H=24, d=128, 880 tokens/frame, chunk 3 frames, window 21 frames, 5 sink "
+    "reference frames, relative RoPE) stacked 30 layers with one rolling cache each; each step is one chunk "
+    "through all 30 layers, 4 denoise reads (fused x0/renoise) + 1 commit per layer"))
 # classifier-free guidance (causal pre-training mode): a second cache per layer for the
 # unconditional branch, 40 guided steps per chunk, guidance scale 5.0
 CFG_CONFIGS = {
@@ -81,6 +90,7 @@ def attention_source_sha256():
 def profiled_traffic(config_name):
     """DRAM bytes per attention launch from the committed ncu record of this workload, if that
     record was taken on the current kernel sources (same sha256), else None."""
+    config_name = {"long": "abot"}.get(config_name, config_name)  # the same launch shape
     rec = os.path.join(ROOT, "profiles", f"chunk_attention_{config_name}.traffic.json")
     if not os.path.exists(rec):
         return None, None
@@ -215,7 +225,8 @@ def run_rkv(args):
     Lq = C * T
     stream = torch.cuda.current_stream()
     sp = stream.cuda_stream
-    h = rkv.RollingKV(1, H, 128, T, W, S, cfg["mode"])
+    n_layers = cfg.get("layers", 1)
+    h = rkv.RollingKV(n_layers, H, 128, T, W, S, cfg["mode"])
     h.set_rope_grid(cfg["gh"], cfg["gw"])
 
     def fill(t, *fields):
@@ -240,33 +251,37 @@ def run_rkv(args):
     state = {"f0": 0}
 
     def step(inp, o=None, x0_buf=None, st=None):
-        """One chunk: four denoise reads with the fused x0 / renoise epilogue, then the commit."""
+        """One chunk through every layer: four denoise reads with the fused x0 / renoise
+        epilogue, then the commit."""
         o = outs if o is None else o
         x0_buf = x0 if x0_buf is None else x0_buf
         st = sp if st is None else st
         f0 = state["f0"]
-        xt = inp["xt"]
-        for s in range(4):
-            sn = SIGMAS[s + 1] if s < 3 else -1.0
-            nxt = xn[s % 2] if sn >= 0 else None
-            h.chunk_attention(0, inp["q"][s], inp["k"][s], inp["v"][s], o[s], C, f0, False, stream=st,
-                              flow=dict(xt=xt, eps=inp["eps"][s] if sn >= 0 else None, sigma=SIGMAS[s],
-                                        sigma_next=sn, x0_out=x0_buf, xt_next_out=nxt))
-            if nxt is not None:
-                xt = nxt
-        h.chunk_attention(0, inp["q"][4], inp["k"][4], inp["v"][4], o[4], C, f0, True, stream=st)
+        for layer in range(n_layers):
+            xt = inp["xt"]
+            for s in range(4):
+                sn = SIGMAS[s + 1] if s < 3 else -1.0
+                nxt = xn[s % 2] if sn >= 0 else None
+                h.chunk_attention(layer, inp["q"][s], inp["k"][s], inp["v"][s], o[s], C, f0, False, stream=st,
+                                  flow=dict(xt=xt, eps=inp["eps"][s] if sn >= 0 else None, sigma=SIGMAS[s],
+                                            sigma_next=sn, x0_out=x0_buf, xt_next_out=nxt))
+                if nxt is not None:
+                    xt = nxt
+            h.chunk_attention(layer, inp["q"][4], inp["k"][4], inp["v"][4], o[4], C, f0, True, stream=st)
         state["f0"] = f0 + C
 
     # reference frames (sinks) and roll the window to steady state
     if cfg["refs"]:
         kr = fill(torch.empty((cfg["refs"] * T, H, 128), **bf), 99, 0, 2)
         vr = fill(torch.empty((cfg["refs"] * T, H, 128), **bf), 99, 0, 3)
-        h.write_chunk(0, kr, vr, cfg["refs"], 0, stream=sp)
+        for layer in range(n_layers):
+            h.write_chunk(layer, kr, vr, cfg["refs"], 0, stream=sp)
         state["f0"] = cfg["refs"]
     prefill = math.ceil((W - S) / C) + 1
     for i in range(prefill):
         inp = pool[i % pool_n]
-        h.chunk_attention(0, inp["q"][4], inp["k"][4], inp["v"][4], outs[4], C, state["f0"], True, stream=sp)
+        for layer in range(n_layers):
+            h.chunk_attention(layer, inp["q"][4], inp["k"][4], inp["v"][4], outs[4], C, state["f0"], True, stream=sp)
         state["f0"] += C
     gpu_id = None
     try:
@@ -284,14 +299,14 @@ def run_rkv(args):
     flops = 0.0
     f = state["f0"]
     for _ in range(args.steps):
-        flops += 5 * 4.0 * H * 128 * Lq * visible_keys(cfg, f, f)
+        flops += n_layers * 5 * 4.0 * H * 128 * Lq * visible_keys(cfg, f, f)
         f += C
 
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     clocks.mark_start()
-    h.timing_begin(5 * args.steps)
+    h.timing_begin(5 * n_layers * args.steps)
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
@@ -300,7 +315,7 @@ def run_rkv(args):
     ev1.record(stream)
     torch.cuda.synchronize()
     clocks.mark_end()
-    kernel_ms = h.timing_end(5 * args.steps)
+    kernel_ms = h.timing_end(5 * n_layers * args.steps)
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
@@ -309,15 +324,17 @@ def run_rkv(args):
     if status != rkv.OK:
         raise RuntimeError("device wait expired in the timed region")
     ms = reduce_max(ms, "cuda")
-    tokens = 5 * Lq * args.steps * world
+    tokens = 5 * n_layers * Lq * args.steps * world
     value = tokens / (ms / 1e3)
 
     # ---- end to end through the C ABI with host buffers (copies inside the timed region)
     e2e = None
-    if not args.no_e2e:
+    # (one layer only: the stacked-layer shape reruns the same kernels, and its layers' inputs
+    # would come from the previous layer on the device, not from the host)
+    if not args.no_e2e and n_layers == 1:
         e2e = run_e2e(args, torch, dist, world, pool, step, tokens)
-    hbm = None if args.no_hbm else measure_hbm_kernels(torch, rkv, synth, cfg, rank)
-    cross = None if args.no_hbm else measure_cross_attention(torch, rkv, synth, cfg, rank)
+    hbm = None if args.no_hbm or n_layers > 1 else measure_hbm_kernels(torch, rkv, synth, cfg, rank)
+    cross = None if args.no_hbm or n_layers > 1 else measure_cross_attention(torch, rkv, synth, cfg, rank)
 
     pk, pk_kind = peaks()
     traffic, traffic_src = profiled_traffic(args.config)
@@ -329,7 +346,8 @@ def run_rkv(args):
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": cfg["workload"], "queries_per_call": Lq, "keys_per_call": W * T,
-                   "calls_per_step": 5, "parallelism": f"replicas x{world} (no data-path collective)",
+                   "calls_per_step": 5 * n_layers, "layers": n_layers,
+                   "parallelism": f"replicas x{world} (no data-path collective)",
                    "l2": f"inputs larger than L2 ({(15 * Lq * H * 128 + 4 * Lq * H * 128) * 2 / 1e6:.0f} MB per step)"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": (achieved / peak) if achieved else None, "traffic": traffic,
@@ -337,11 +355,11 @@ def run_rkv(args):
                      "kernel": "chunk_attention_kernel", "peak_source": f"{pk_kind} bf16_tflops_sustained",
                      "frac_of_burst": (achieved / pk["bf16_tflops"]) if achieved else None,
                      "mean_kernel_ms": mean_kernel_ms, "launches_timed": len(kernel_ms),
-                     "flops_per_launch": flops / max(1, 5 * args.steps)},
+                     "flops_per_launch": flops / max(1, 5 * n_layers * args.steps)},
         "e2e": e2e,
         "hbm_kernels": hbm,
         "cross_attention": cross,
-        "gpu_launches": 11 * args.steps,
+        "gpu_launches": 11 * n_layers * args.steps,
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
