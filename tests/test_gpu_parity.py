@@ -90,6 +90,10 @@ SMALL = [
     Config("tiny-slots-refs", 8, H=2, grid_h=4, grid_w=4, C=2, W=6, S=2, rope_mode=SLOTS, refs=2, chunks=10),
     Config("ragged-slots", 9, H=3, grid_h=8, grid_w=10, C=3, W=7, S=2, rope_mode=SLOTS, refs=1, chunks=8, reads=2),
     Config("straddle-slots", 10, H=2, grid_h=4, grid_w=6, C=4, W=18, S=6, rope_mode=SLOTS, chunks=8, reads=1),
+    # the chunk fills the whole ring (W - S == C): no history frame is ever visible
+    Config("no-history", 11, H=2, grid_h=4, grid_w=6, C=3, W=4, S=1, rope_mode=ABS, chunks=6, reads=1),
+    # the largest window the library takes (256 frames), filled and then evicting
+    Config("max-window", 12, H=1, grid_h=2, grid_w=8, C=4, W=256, S=3, rope_mode=REL, chunks=70, reads=1),
 ]
 
 
