@@ -127,9 +127,10 @@ __device__ __forceinline__ uint4 flow_x0(const FlowStep& step, double scale, uin
 
 // One 16-byte vector of each operand per thread per iteration. The bf16 <-> fp64
 // conversions run on the special-function unit and keep it busy, so HBM stays busy only
-// with many resident warps: few registers per thread (40) and a grid of 16 blocks per SM.
+// with many resident warps: 32 registers per thread (eight blocks of 256 threads per SM)
+// and a grid of 16 blocks per SM.
 template <bool kCfg>
-__global__ void __launch_bounds__(256) flow_kernel(const FlowParams p) {
+__global__ void __launch_bounds__(256, 8) flow_kernel(const FlowParams p) {
   FlowStep step;
   step.sigma = p.sigma;
   step.renoise = p.sigma_next >= 0.0;
