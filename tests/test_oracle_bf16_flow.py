@@ -49,6 +49,20 @@ def test_bf16_to_f64_known_values():
     assert bf16.to_f64(np.array([0x7F7F]))[0] == (2 - 2 ** -7) * 2.0 ** 127
 
 
+def test_bf16_overflow_boundary():
+    """IEEE 754 round-to-nearest-even overflow: the largest finite bf16 is (2 - 2^-7) 2^127
+    (0x7F7F); everything below the midpoint (2 - 2^-8) 2^127 to the next power 2^128 rounds
+    down to it, the midpoint ties to the even neighbour 2^128, which is out of range, and
+    becomes infinity, as does everything above it."""
+    top = (2 - 2 ** -7) * 2.0 ** 127
+    mid = (2 - 2 ** -8) * 2.0 ** 127
+    below = np.nextafter(mid, 0.0)
+    for x, want in [(top, 0x7F7F), (below, 0x7F7F), (mid, 0x7F80), (np.nextafter(mid, np.inf), 0x7F80),
+                    (1e39, 0x7F80), (-below, 0xFF7F), (-mid, 0xFF80), (-top, 0xFF7F), (-1e300, 0xFF80)]:
+        got = int(bf16.from_f64(np.array([x]))[0])
+        assert got == want, (x, hex(got), hex(want))
+
+
 def test_bf16_nearest_by_brute_force():
     rng = np.random.default_rng(1)
     x = rng.standard_normal(20000) * np.exp(rng.uniform(-30, 30, 20000))

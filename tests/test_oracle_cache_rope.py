@@ -4,7 +4,8 @@ Cache: a hand-worked fixture, the closed form of what a window of W frames with
 S sinks holds after n in-order frames, the ring-slot closed form, and the
 "sinks never move" invariant. RoPE: an independent complex-exponential
 formulation, the identity at position 0, the 1-radian special case, norm
-preservation, and the relative-position property of the scores.
+preservation, the relative-position property of the scores, and the time ids of the
+standalone rotation in relative mode against a hand-worked list.
 """
 import cmath
 import math
@@ -13,8 +14,9 @@ import os
 import numpy as np
 import pytest
 
-from oracle import rope
+from oracle import bf16, rope
 from oracle.cache import CapacityError, RollingCache
+from oracle.layer import OracleLayer
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -198,6 +200,26 @@ def test_relative_time_ids():
     ids = rope.time_ids_relative(frames, f0, C, W)
     assert list(ids) == [0] * S + list(range(S, W - C)) + [18, 19, 20]
     assert ids.min() >= 0 and ids.max() <= W - 1
+
+
+def test_rope_apply_relative_ids_hand_worked():
+    # standalone rotation, relative mode: t = clamp(f - (window_end - W), 0, W - 1), W = 6
+    H, gh, gw, W, S, D = 1, 1, 2, 6, 2, 128
+    T = gh * gw
+    lay = OracleLayer(H, D, T, gh, gw, W, S, OracleLayer.RELATIVE)
+    rng = np.random.default_rng(6)
+    cases = [
+        (10, 2, 12, [4, 5]),        # the window's last two frames
+        (0, 2, 12, [0, 0]),         # old sinks clamp to 0
+        (6, 4, 12, [0, 1, 2, 3]),
+        (0, 4, 4, [2, 3, 4, 5]),    # warm-up: the window end is frame 4
+        (40, 2, 30, [5, 5]),        # beyond the window end: clamped to W - 1
+    ]
+    for start, n, end, ids in cases:
+        x = bf16.from_f64(rng.standard_normal((n * T, H, D)))
+        got = lay.rope_apply(x, n, start, end)
+        want = rope.rotate(bf16.to_f64(x), rope.token_positions(ids, T, gw))
+        assert np.array_equal(got, want), (start, n, end)
 
 
 def test_token_positions_grid_order():
