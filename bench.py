@@ -775,6 +775,77 @@ def run_reference(args):
     }), flush=True)
 
 
+def run_isolated(args):
+    """A few launches of one kernel at the workload's sizes and nothing else, for profiler
+    captures (``ncu -k <kernel> -s 1 -c 1 python bench.py --isolate ...``): ``commit``
+    (rkv_write_chunk: the ring write-back), ``rope`` (rkv_rope_apply of one chunk's
+    [Lq, H, 128] tensor), ``flow`` (rkv_flow_x0_renoise on the [Lq, H*128] latent, renoise
+    on) or ``cross`` (rkv_cross_attention of the chunk's queries over 512 text tokens).
+    Launches rotate over buffer sets that together exceed the 126 MB L2. Prints one JSON line
+    with the mean CUDA-event time per launch (not a benchmark line)."""
+    import torch
+    import rolling_kv_chunked_b200 as rkv
+    import synth
+    cfg = CONFIGS[args.config]
+    H, C, W, S = cfg["H"], cfg["C"], cfg["W"], cfg["S"]
+    T = cfg["gh"] * cfg["gw"]
+    Lq = C * T
+    n = Lq * H * 128
+    st = torch.cuda.current_stream()
+    sp = st.cuda_stream
+    bf = dict(dtype=torch.bfloat16, device="cuda")
+
+    def fill(t, *f):
+        synth.fill_normal_bf16_cuda(t.data_ptr(), t.numel(), synth.stream_key(0, 91, *f), 0, sp)
+        return t
+
+    per_set = {"commit": 2, "rope": 1, "flow": 5, "cross": 2}[args.isolate]
+    n_sets = max(2, -(-int(256e6) // (per_set * n * 2)))
+    sets = [[fill(torch.empty((Lq, H, 128), **bf), i, j) for j in range(per_set)] for i in range(n_sets)]
+    h = None
+    if args.isolate in ("commit", "rope", "cross"):
+        h = rkv.RollingKV(1, H, 128, T, W, S, cfg["mode"])
+        h.set_rope_grid(cfg["gh"], cfg["gw"])
+    if args.isolate == "commit":
+        state = {"f": 0}
+
+        def launch(b):
+            h.write_chunk(0, b[0], b[1], C, state["f"], stream=sp)
+            state["f"] += C
+        work = {"bytes_per_launch": 8 * n + (4 * n if cfg["mode"] == 0 else 0)}
+    elif args.isolate == "rope":
+        def launch(b):
+            h.rope_apply(b[0], C, 0, C, stream=sp)
+        work = {"bytes_per_launch": 4 * n}
+    elif args.isolate == "flow":
+        def launch(b):
+            lat = [x.view(Lq, H * 128) for x in b]
+            rkv.flow_x0_renoise(lat[0], lat[1], lat[2], 1.0, 0.75, lat[3], lat[4], stream=sp)
+        work = {"bytes_per_launch": 10 * n}
+    else:
+        n_text = 512
+        h.set_text_kv(0, fill(torch.empty((n_text, H, 128), **bf), 1000), fill(torch.empty((n_text, H, 128), **bf), 1001),
+                      stream=sp)
+
+        def launch(b):
+            h.cross_attention(0, b[0], b[1], stream=sp)
+        work = {"flops_per_launch": 4.0 * H * 128 * Lq * n_text}
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * args.reps)]
+    torch.cuda.synchronize()
+    for i in range(args.reps):
+        ev[2 * i].record(st)
+        launch(sets[i % n_sets])
+        ev[2 * i + 1].record(st)
+    torch.cuda.synchronize()
+    if h is not None:
+        if h.poll_device_status(sp) != rkv.OK:
+            raise RuntimeError("device wait expired")
+        h.close()
+    us = [ev[2 * i].elapsed_time(ev[2 * i + 1]) * 1e3 for i in range(args.reps)]
+    print(json.dumps({"isolate": args.isolate, "config": args.config, "launches": args.reps,
+                      "us_per_launch": us, **work}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -787,7 +858,15 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end pass")
     ap.add_argument("--no-hbm", action="store_true",
                     help="skip the side measurements (HBM-bound kernels, cross-attention)")
+    ap.add_argument("--isolate", choices=["commit", "rope", "flow", "cross"],
+                    help="only launch this kernel --reps times at the config's sizes (for profiler captures)")
+    ap.add_argument("--reps", type=int, default=3, help="launches of the --isolate kernel")
     args = ap.parse_args()
+    if args.isolate:
+        if args.config not in CONFIGS:
+            ap.error("--isolate takes one of " + ", ".join(sorted(CONFIGS)))
+        run_isolated(args)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
