@@ -41,15 +41,15 @@ CONFIGS = {
     "abot": dict(workload="ABot-style relative RoPE: 1 layer, H=24, d=128, 880 tokens/frame (22x40 grid), "
                           "chunk 3 frames (2640 queries), window 21 frames (18480 keys), 5 sink reference frames, "
                           "4 denoise reads (fused x0/renoise) + 1 commit per chunk",
-                 H=24, gh=22, gw=40, C=3, W=21, S=5, refs=5, mode=1),
+                 H=24, gh=22, gw=40, C=3, W=21, S=5, refs=5, mode=1, rollout_chunks=64),
     "480p": dict(workload="LingBot-style 480P: 1 layer, H=40, d=128, 1560 tokens/frame (30x52 grid), chunk 4 frames "
                           "(6240 queries), window 18 frames (28080 keys), sink 6, absolute RoPE, "
                           "4 denoise reads (fused x0/renoise) + 1 commit per chunk",
-                 H=40, gh=30, gw=52, C=4, W=18, S=6, refs=0, mode=0),
+                 H=40, gh=30, gw=52, C=4, W=18, S=6, refs=0, mode=0, rollout_chunks=22),
     "720p": dict(workload="720p: 1 layer, H=40, d=128, 3600 tokens/frame (45x80 grid), chunk 4 frames (14400 queries), "
                           "window 18 frames (64800 keys), sink 6, absolute RoPE, fused x0/renoise on the "
                           "[14400 x 5120] latent, 4 denoise reads + 1 commit per chunk",
-                 H=40, gh=45, gw=80, C=4, W=18, S=6, refs=0, mode=0),
+                 H=40, gh=45, gw=80, C=4, W=18, S=6, refs=0, mode=0, rollout_chunks=30),
 }
 # the long-rollout stress shape: the ABot layer stacked 30 deep, one rolling cache per layer,
 # every step = one chunk through all layers (the layers reuse one seeded input set per call;
@@ -327,6 +327,30 @@ def run_rkv(args):
     tokens = 5 * n_layers * Lq * args.steps * world
     value = tokens / (ms / 1e3)
 
+    # ---- a whole rollout from an empty cache: the reference frames, then every chunk of the
+    # workload's video (4 reads + 1 commit each), warm-up chunks with short windows included
+    rollout = None
+    if n_layers == 1 and world == 1 and not args.no_rollout:
+        h.reset()
+        state["f0"] = 0
+        r0 = torch.cuda.Event(enable_timing=True)
+        r1 = torch.cuda.Event(enable_timing=True)
+        r0.record(stream)
+        if cfg["refs"]:
+            h.write_chunk(0, kr, vr, cfg["refs"], 0, stream=sp)
+            state["f0"] = cfg["refs"]
+        n_chunks = cfg["rollout_chunks"]
+        for i in range(n_chunks):
+            step(pool[i % pool_n])
+        r1.record(stream)
+        torch.cuda.synchronize()
+        if h.poll_device_status(sp) != rkv.OK:
+            raise RuntimeError("device wait expired in the rollout")
+        r_ms = r0.elapsed_time(r1)
+        rollout = {"chunks": n_chunks, "frames": n_chunks * C, "ms": r_ms,
+                   "query_tokens_per_s": 5 * n_chunks * Lq / (r_ms / 1e3),
+                   "frames_per_s": n_chunks * C / (r_ms / 1e3)}
+
     # ---- end to end through the C ABI with host buffers (copies inside the timed region)
     e2e = None
     # (one layer only: the stacked-layer shape reruns the same kernels, and its layers' inputs
@@ -356,6 +380,8 @@ def run_rkv(args):
                      "frac_of_burst": (achieved / pk["bf16_tflops"]) if achieved else None,
                      "mean_kernel_ms": mean_kernel_ms, "launches_timed": len(kernel_ms),
                      "flops_per_launch": flops / max(1, 5 * n_layers * args.steps)},
+        "frames_per_s_per_layer": C * n_layers * args.steps * world / (ms / 1e3),
+        "rollout": rollout,
         "e2e": e2e,
         "hbm_kernels": hbm,
         "cross_attention": cross,
@@ -858,6 +884,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end pass")
     ap.add_argument("--no-hbm", action="store_true",
                     help="skip the side measurements (HBM-bound kernels, cross-attention)")
+    ap.add_argument("--no-rollout", action="store_true", help="skip the whole-rollout pass")
     ap.add_argument("--isolate", choices=["commit", "rope", "flow", "cross"],
                     help="only launch this kernel --reps times at the config's sizes (for profiler captures)")
     ap.add_argument("--reps", type=int, default=3, help="launches of the --isolate kernel")
