@@ -26,8 +26,11 @@
 // product straight from TMEM. MMA issue order per key tile j:
 //   S0(j) = Q0 K_j^T, PV1(j-1), S1(j) = Q1 K_j^T, PV0(j)
 // so that while one softmax warpgroup works on its tile the tensor core runs the
-// other tile's products. Online softmax in the log2 domain against a running reference:
-// each thread reads its S row once (64 columns at a time) and forms the numerators
+// other tile's products. PV0(j) -> S0(j+1) is query tile 0's critical chain, so the
+// issuer observes V(j) and probes K(j+1) before it waits for P0(j) (where it is idle):
+// nothing but that wait stands between P0(j) and the 16 products PV0(j), S0(j+1).
+// Online softmax in the log2 domain against a running reference: each thread reads its
+// S row once (64 columns at a time) and forms the numerators
 // 2^(s/sqrt(d) log2 e - reference) directly; the tile's numerator sum both feeds the row
 // sum and bounds the tile's largest numerator, so the reference moves (and O is rescaled,
 // at the start of the next tile) only when that sum exceeds 2^8, and a sum above 2^64
@@ -313,10 +316,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < kHeadDim / 16; ++kk)
           ptx::mma_ss(tmem + col_s(t), desc_kmajor(q_addr[t], kk), desc_kmajor(kt, kk), kIdescS, kk > 0 ? 1u : 0u);
       };
-      // O_t += P_t(jj) V(jj); returns false if a wait expired
+      // O_t += P_t(jj) V(jj) with V(jj) already observed; returns false if a wait expired
       auto issue_pv = [&](int t, int jj) -> bool {
         if (!ptx::mbar_wait(&bars[kBarPFull + t], jj & 1, limit)) return false;
-        if (!ptx::mbar_wait(&bars[kBarVFull + (jj & 1)], (jj >> 1) & 1, limit)) return false;
         ptx::tc_fence_after();
         const uint32_t vt = v_addr + (jj & 1) * kTile;
 #pragma unroll
@@ -327,9 +329,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
 
+      // The waits on K(j+1) and V(j) are taken before the wait for P0(j), where this thread is
+      // idle anyway, so that PV0(j) and S0(j+1) follow P0(j) with no other wait between them.
+      bool k_ready = ok && ptx::mbar_wait(&bars[kBarKFull + 0], 0, limit);
+      if (!k_ready) ok = false;
       for (int j = 0; ok && j < n_tiles; ++j) {
         const int s = j & 1;
-        if (!ptx::mbar_wait(&bars[kBarKFull + s], (j >> 1) & 1, limit)) { ok = false; break; }
+        if (!k_ready && !ptx::mbar_wait(&bars[kBarKFull + s], (j >> 1) & 1, limit)) { ok = false; break; }
         ptx::tc_fence_after();
         const uint32_t kt = k_addr + s * kTile;
         issue_s(0, kt);
@@ -338,6 +344,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue_s(1, kt);
         ptx::mma_commit(&bars[kBarSFull + 1]);
         ptx::mma_commit(&bars[kBarKEmpty + s]);
+        if (!ptx::mbar_wait(&bars[kBarVFull + s], (j >> 1) & 1, limit)) { ok = false; break; }
+        k_ready = j + 1 < n_tiles && ptx::mbar_try_wait(&bars[kBarKFull + (s ^ 1)], ((j + 1) >> 1) & 1);
         if (!issue_pv(0, j)) { ok = false; break; }
       }
       if (ok && !issue_pv(1, n_tiles - 1)) ok = false;
