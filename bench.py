@@ -766,9 +766,19 @@ def cpu_baseline(cfg, budget_s=10.0, heads=2):
         if el >= budget_s:
             break
     per_call_s = el / n * (H / heads)
+    # the oracle's x0 / renoise step (K4) on an eighth of the workload's latent
+    from oracle import flow as oflow
+    import synth
+    n_el = C * T * H * 128 // 8
+    xt, v, eps = (synth.normal_bf16_bits(synth.stream_key(0, 93, i), 0, n_el) for i in range(3))
+    t1 = time.perf_counter()
+    oflow.x0_renoise_bf16(xt, v, eps, 1.0, 0.75)
+    flow_s = time.perf_counter() - t1
     return {"value": C * T / per_call_s, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
             "sample": f"{n} steady-state reads x {heads} of {H} heads (all {C * T} queries vs {cfg['W'] * T} keys), "
-                      f"numpy fp64, scaled by {H}/{heads}"}
+                      f"numpy fp64, scaled by {H}/{heads}",
+            "flow_x0_renoise": {"GB/s": 10 * n_el / flow_s / 1e9, "elements": n_el,
+                                "sample": "one call on an eighth of the latent, sigma 1.0 -> 0.75, numpy fp64"}}
 
 
 def run_reference(args):
