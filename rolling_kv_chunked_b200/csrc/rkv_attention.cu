@@ -35,7 +35,7 @@
 // sum and bounds the tile's largest numerator, so the reference moves (and O is rescaled,
 // at the start of the next tile) only when that sum exceeds 2^8, and a sum above 2^64
 // sends the warp to an exact path that takes the row maximum first (always used for the
-// first tile). Exponentials run on the special-function unit, one pair in eight on the
+// first tile). Exponentials run on the special-function unit, two pairs in eight on the
 // FMA pipe as a polynomial; P is rounded to bf16 (nearest even) in pairs.
 //
 // Every mbarrier wait is bounded in wall time; on expiry the kernel records
@@ -156,7 +156,7 @@ __device__ __forceinline__ void exp2_poly_x2(uint64_t x2, float& y0, float& y1) 
 // row sums (of the unrounded values) accumulate in acc.
 // kPoly: kPolyPairs of every 8 pairs take the polynomial path (full tiles only).
 #ifndef RKV_POLY_PAIRS
-#define RKV_POLY_PAIRS 1
+#define RKV_POLY_PAIRS 2
 #endif
 constexpr int kPolyPairs = RKV_POLY_PAIRS;
 template <bool kPoly>
