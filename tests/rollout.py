@@ -34,6 +34,9 @@ class Config:
     S: int
     rope_mode: int
     refs: int = 0          # reference frames written with write_chunk before the chunks (become sinks)
+    # compare with the oracle's output rounded to bf16 (shapes with a handful of visible keys,
+    # whose O(1) outputs put bf16's own rounding at the size of the mean bound)
+    ref_bf16: bool = False
     chunks: int = 4
     reads: int = 4
     layers: int = 1
@@ -78,7 +81,28 @@ def compare(out_bits: np.ndarray, ref: np.ndarray):
     return float(err.max()), float(err.mean()), rel
 
 
-def assert_close(out_bits, ref, what=""):
+def bf16_ulp(x: np.ndarray) -> np.ndarray:
+    """Spacing of the bf16 values at |x| (normal range): 2^(floor(log2 |x|) - 7)."""
+    e = np.floor(np.log2(np.maximum(np.abs(x), 2.0 ** -126)))
+    return np.ldexp(1.0, (e - 7).astype(np.int64))
+
+
+def assert_close(out_bits, ref, what="", ref_bf16=False):
+    """The tolerance of the attention outputs. With ref_bf16 (shapes where a query sees only a
+    few keys, so the outputs are of order one) the oracle's value is first rounded to bf16
+    (nearest even), since the format's own rounding of the exact value averages about 2^-9 of
+    it, the size of the mean bound; and an element may then differ from that rounded value by
+    one bf16 step at its magnitude when that step exceeds the absolute bound (outputs of 2 and
+    more)."""
+    if ref_bf16:
+        ref = bf16.to_f64(bf16.from_f64(ref))
+        got = bf16.to_f64(out_bits)
+        allowed = np.maximum(MAX_ABS, bf16_ulp(ref))
+        bad = np.abs(got - ref) > allowed
+        assert not bad.any(), f"{what}: {int(bad.sum())} elements beyond max(1.5e-2, one bf16 step)"
+        mx, mean, rel = compare(out_bits, ref)
+        assert mean <= MEAN_ABS and rel <= REL_RMS, f"{what}: max {mx:.3e} mean {mean:.3e} rel {rel:.3e}"
+        return mx, mean, rel
     mx, mean, rel = compare(out_bits, ref)
     assert mx <= MAX_ABS and mean <= MEAN_ABS and rel <= REL_RMS, f"{what}: max {mx:.3e} mean {mean:.3e} rel {rel:.3e}"
     return mx, mean, rel
@@ -164,7 +188,7 @@ class Rollout:
                 got = got[np.asarray(rows)]
             if heads is not None:
                 got = got[:, np.asarray(heads)]
-            r = assert_close(got, ref, f"{c.name} layer {layer} chunk {chunk} call {call}")
+            r = assert_close(got, ref, f"{c.name} layer {layer} chunk {chunk} call {call}", c.ref_bf16)
             if stats is not None:
                 stats.append(r)
         self.f0[layer] = f0 + c.C

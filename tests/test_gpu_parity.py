@@ -94,6 +94,13 @@ SMALL = [
     Config("no-history", 11, H=2, grid_h=4, grid_w=6, C=3, W=4, S=1, rope_mode=ABS, chunks=6, reads=1),
     # the largest window the library takes (256 frames), filled and then evicting
     Config("max-window", 12, H=1, grid_h=2, grid_w=8, C=4, W=256, S=3, rope_mode=REL, chunks=70, reads=1),
+    # one-token frames: one query row per chunk, every key segment a one-key ragged tile; with
+    # 1-5 visible keys the outputs are of order one, so they are compared with the oracle's
+    # output rounded to bf16
+    Config("single-token", 13, H=2, grid_h=1, grid_w=1, C=1, W=4, S=1, rope_mode=REL, chunks=8, reads=1,
+           ref_bf16=True),
+    Config("single-token-abs", 14, H=3, grid_h=1, grid_w=1, C=2, W=5, S=2, rope_mode=ABS, chunks=8, reads=2,
+           ref_bf16=True),
 ]
 
 
