@@ -86,8 +86,13 @@ class OracleLayer:
         return [f.frame for f in self.cache.after_append(ids)]
 
     def chunk_attention(self, q_bits, k_bits, v_bits, n_frames, start_frame, commit,
-                        rows=None, heads=None):
-        """fp64 attention output [len(rows), len(heads), d] for the chunk's queries."""
+                        rows=None, heads=None, rope_out_bf16=False):
+        """fp64 attention output [len(rows), len(heads), d] for the chunk's queries.
+
+        rope_out_bf16: round the rotated queries and keys to bf16 (nearest even) before the
+        attention, as the pages' bf16 pipeline hands them over ([P2] §3: causal_rope_apply's
+        bf16 output goes into attention(roped_query, k_cache, v_cache)); off by default (the
+        rotation stays exact in fp64)."""
         self._check_order(start_frame)
         chunk = self._split_frames(k_bits, v_bits, n_frames, start_frame)
         window = self.cache.after_append(chunk)
@@ -112,6 +117,9 @@ class OracleLayer:
             rows = np.asarray(rows)
             q, q_pos = q[rows], q_pos[rows]
         q_rot = rope.rotate(bf16.to_f64(q), q_pos, self.theta, self.pairs)
+        if rope_out_bf16:
+            q_rot = bf16.to_f64(bf16.from_f64(q_rot))
+            k_rot = bf16.to_f64(bf16.from_f64(k_rot))
 
         out = attend(q_rot, k_rot, bf16.to_f64(v))
         if commit:

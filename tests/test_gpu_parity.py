@@ -101,6 +101,11 @@ SMALL = [
            ref_bf16=True),
     Config("single-token-abs", 14, H=3, grid_h=1, grid_w=1, C=2, W=5, S=2, rope_mode=ABS, chunks=8, reads=2,
            ref_bf16=True),
+    # a peaked softmax: queries x 4 (scores x 4), through warm-up, eviction and wrap
+    Config("peaked-rel", 15, H=2, grid_h=8, grid_w=10, C=3, W=7, S=2, rope_mode=REL, refs=1, chunks=8, reads=1,
+           q_scale=4.0),
+    Config("peaked-abs", 16, H=2, grid_h=10, grid_w=20, C=2, W=5, S=1, rope_mode=ABS, chunks=6, reads=1,
+           q_scale=4.0),
 ]
 
 

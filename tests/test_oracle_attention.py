@@ -112,6 +112,38 @@ def test_rolling_equals_explicit_mask_when_window_covers_history(mode, tol):
         frames += list(range(f0, f0 + C))
 
 
+def test_rope_out_bf16_rounds_the_rotated_operands():
+    """rope_out_bf16: the attention of the rotated queries and keys rounded to bf16, pinned with
+    the independent complex-exponential rotation and full masked attention (absolute ids, a
+    window that covers all history); scores x 4 so that the rounding visibly changes the result."""
+    H, d, gh, gw, C, S, n_chunks = 2, 128, 2, 2, 2, 2, 3
+    T = gh * gw
+    W = C * n_chunks + 2
+    lay = OracleLayer(H, d, T, gh, gw, W, S, OracleLayer.ABSOLUTE)
+    rng = np.random.default_rng(23)
+    committed_k, committed_v = [], []
+    for c in range(n_chunks):
+        f0 = c * C
+        q, k, v = _bits(rng, (C * T, H, d), 4.0), _bits(rng, (C * T, H, d)), _bits(rng, (C * T, H, d))
+        unrounded = lay.chunk_attention(q, k, v, C, f0, commit=False)   # a read: no state change
+        out = lay.chunk_attention(q, k, v, C, f0, commit=True, rope_out_bf16=True)
+        assert np.max(np.abs(unrounded - out)) > 1e-4   # the rounding visibly changes the result
+        k_all = np.concatenate(committed_k + [bf16.to_f64(k)], axis=0)
+        v_all = np.concatenate(committed_v + [bf16.to_f64(v)], axis=0)
+        frames = list(range(f0 + C))
+        qr = bf16.to_f64(bf16.from_f64(_rot_complex(bf16.to_f64(q), list(range(f0, f0 + C)), T, gw)))
+        kr = bf16.to_f64(bf16.from_f64(_rot_complex(k_all, frames, T, gw)))
+        ref = np.empty_like(out)
+        for h in range(H):
+            sc = qr[:, h, :] @ kr[:, h, :].T / math.sqrt(d)
+            sc -= sc.max(axis=1, keepdims=True)
+            pw = np.exp(sc)
+            ref[:, h, :] = (pw / pw.sum(axis=1, keepdims=True)) @ v_all[:, h, :]
+        assert np.max(np.abs(out - ref)) < 1e-12, c
+        committed_k.append(bf16.to_f64(k))
+        committed_v.append(bf16.to_f64(v))
+
+
 # ----------------------------------------------------------------- visible set closed form
 def _visible_frames(f0, C, W, S):
     R = W - S
