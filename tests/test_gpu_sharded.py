@@ -4,7 +4,8 @@ Each emulated rank is a HeadShardedRollingKV (its own caches of H/2 heads); the 
 with this library's kernels (rkv_copy_heads packs / unpacks the head blocks, the chunk
 attention runs per rank) and the all-to-all between the ranks is done in-process by the
 test (copies of the ranks' send slices; no collective, nothing waits on another rank).
-Checked against one unsharded RollingKV of all heads on the same inputs: every output
+Checked against one unsharded RollingKV of all heads on the same inputs, at a small shape and
+at the ABot shape (24 heads, 880 tokens per frame, window 21 with 5 sinks): every output
 block bit for bit, through sinks, warm-up, eviction and wrap, both RoPE modes, and the x0 /
 renoise step on each rank's latent block bit for bit against the unsharded fused epilogue;
 the caches of each rank equal the unsharded cache's heads bit for bit; rkv_copy_heads
@@ -25,8 +26,10 @@ if not torch.cuda.is_available():
 import rolling_kv_chunked_b200 as rkv  # noqa: E402
 from rolling_kv_chunked_b200.sharded import HeadShardedRollingKV  # noqa: E402
 
-H, GH, GW, C, W, S, G = 4, 8, 10, 2, 6, 2, 2
-T = GH * GW
+G = 2
+# (H, grid_h, grid_w, C, W, S, chunks): a small shape, and the ABot shape through its first
+# evictions (window 21 frames with 5 sinks, chunks of 3 frames of 22 x 40 tokens)
+SHAPES = {"small": (4, 8, 10, 2, 6, 2, 5), "abot": (24, 22, 40, 3, 21, 5, 7)}
 
 
 def _dev(key, shape):
@@ -40,7 +43,7 @@ def _exchange(sends):
     return [torch.stack([sends[i][j] for i in range(G)]) for j in range(G)]
 
 
-def _sharded_call(ranks, *tensors, n_frames):
+def _sharded_call(ranks, H, *tensors, n_frames):
     """Pack each rank's token blocks, exchange, and return every rank's [Lq, H/G, d] inputs."""
     per_rank = []
     for x in tensors:
@@ -49,8 +52,11 @@ def _sharded_call(ranks, *tensors, n_frames):
     return per_rank
 
 
+@pytest.mark.parametrize("shape", sorted(SHAPES))
 @pytest.mark.parametrize("mode", [rkv.ROPE_ABSOLUTE, rkv.ROPE_RELATIVE])
-def test_two_emulated_ranks_match_unsharded_bit_for_bit(mode):
+def test_two_emulated_ranks_match_unsharded_bit_for_bit(mode, shape):
+    H, GH, GW, C, W, S, n_chunks = SHAPES[shape]
+    T = GH * GW
     ranks = [HeadShardedRollingKV(1, H, 128, T, W, S, mode, world_size=G, rank=r) for r in range(G)]
     full = rkv.RollingKV(1, H, 128, T, W, S, mode)
     for h in ranks + [full]:
@@ -64,13 +70,13 @@ def test_two_emulated_ranks_match_unsharded_bit_for_bit(mode):
 
     # sinks written without attention
     kr, vr = _dev(synth.stream_key(6, 1), (S * T, H, 128)), _dev(synth.stream_key(6, 2), (S * T, H, 128))
-    (k_in, v_in) = _sharded_call(ranks, blocks(kr, S * T), blocks(vr, S * T), n_frames=S)
+    (k_in, v_in) = _sharded_call(ranks, H, blocks(kr, S * T), blocks(vr, S * T), n_frames=S)
     for r in range(G):
         ranks[r].local.write_chunk(0, k_in[r], v_in[r], S, 0)
     full.write_chunk(0, kr, vr, S, 0)
     f0 = S
     sig = [1.0, 0.75]
-    for chunk in range(5):
+    for chunk in range(n_chunks):
         xt = _dev(synth.stream_key(6, 3, chunk), (Lq, H * 128))
         for call in range(2):
             commit = call == 1
@@ -84,7 +90,7 @@ def test_two_emulated_ranks_match_unsharded_bit_for_bit(mode):
                 full.chunk_attention(0, q, k, v, out_full, C, f0, False,
                                      flow=dict(xt=xt, eps=eps, sigma=sig[0], sigma_next=sig[1],
                                                x0_out=x0_full, xt_next_out=xn_full))
-            qs, ks, vs = _sharded_call(ranks, blocks(q, Lq), blocks(k, Lq), blocks(v, Lq), n_frames=C)
+            qs, ks, vs = _sharded_call(ranks, H, blocks(q, Lq), blocks(k, Lq), blocks(v, Lq), n_frames=C)
             outs_h = [ranks[r].attend(0, qs[r], ks[r], vs[r], C, f0, commit) for r in range(G)]
             back = _exchange([o.view(G, Lb, H // G, 128) for o in outs_h])
             for r in range(G):
