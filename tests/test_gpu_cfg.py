@@ -18,7 +18,7 @@ import pytest
 import synth
 from oracle import flow as oflow
 from oracle.layer import OracleLayer
-from rollout import Config, Rollout, assert_close, dev_tensor, host_bits, to_bits
+from rollout import Config, Rollout, assert_close, dev_tensor, host_bits, sample_rows, to_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -163,3 +163,63 @@ def test_cfg_argument_errors_launch_nothing():
     torch.cuda.synchronize()
     assert h.frames_committed(0) == cfg.C and h.poll_device_status() == rkv.OK
     h.close()
+
+
+def test_cfg_fused_epilogue_abot_size():
+    """The guided mode at the ABot shape (24 heads, 2640 queries, 18480 keys, relative RoPE,
+    five reference sinks): two caches, 7 chunks of 4 guided steps, through the first evictions.
+    On the chunks after evictions start: the fused guided x0 / renoise outputs bit for bit
+    against the oracle's epilogue on the stored bf16 c and u, and both branches' attention on
+    sampled rows of the first and last head; both caches bit for bit at the end."""
+    cfg = Config("cfg-abot", 25, H=24, grid_h=22, grid_w=40, C=3, W=21, S=5, rope_mode=REL, refs=5, chunks=7,
+                 reads=4)
+    steps = 4
+    branches = [Rollout(cfg, rkv, torch), Rollout(replace(cfg, seed=cfg.seed + 1), rkv, torch)]
+    Lq, n = cfg.Lq, cfg.Lq * cfg.H * 128
+    sig = _schedule(steps)
+    rows, heads = sample_rows(Lq, n=64, seed=25), [0, cfg.H - 1]
+    checked = {5, 6}
+    outs = [torch.empty((Lq, cfg.H, 128), dtype=torch.bfloat16, device="cuda") for _ in branches]
+    for chunk in range(cfg.chunks):
+        f0 = branches[0].f0[0]
+        xt = _dev_bits(synth.stream_key(cfg.seed, cfg.cfg_id, 99, chunk), n)
+        xt_ref = to_bits(xt) if chunk in checked else None
+        for step in range(steps):
+            s, sn = sig[step], sig[step + 1]
+            eps = _dev_bits(synth.stream_key(cfg.seed, cfg.cfg_id, 98, chunk, step), n)
+            x0 = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+            xn = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+            qkv = [[dev_tensor(torch, b.cfg, 0, chunk, step, t, Lq) for t in "qkv"] for b in branches]
+            branches[0].h.chunk_attention(0, *qkv[0], outs[0], cfg.C, f0, False)
+            branches[1].h.chunk_attention(0, *qkv[1], outs[1], cfg.C, f0, False,
+                                          flow=dict(xt=xt, eps=eps, sigma=s, sigma_next=sn, x0_out=x0,
+                                                    xt_next_out=xn if sn >= 0 else None,
+                                                    v_cond=outs[0], cfg_scale=CFG_SCALE))
+            torch.cuda.synchronize()
+            if chunk not in checked:
+                if sn >= 0:
+                    xt = xn
+                continue
+            c_bits, u_bits = to_bits(outs[0]), to_bits(outs[1])
+            rx0, rxn = oflow.cfg_x0_renoise_bf16(xt_ref, c_bits.reshape(-1), u_bits.reshape(-1), to_bits(eps),
+                                                 CFG_SCALE, s, sn)
+            assert np.array_equal(to_bits(x0), rx0), (chunk, step)
+            if sn >= 0:
+                assert np.array_equal(to_bits(xn), rxn), (chunk, step)
+                xt, xt_ref = xn, rxn
+            if step == 0:
+                for b, got in zip(branches, (c_bits, u_bits)):
+                    ref = b.oracles[0].chunk_attention(*(host_bits(b.cfg, 0, chunk, step, t, Lq) for t in "qkv"),
+                                                       cfg.C, f0, False, rows=rows, heads=heads)
+                    assert_close(got[rows][:, heads], ref, f"{b.cfg.name} seed {b.cfg.seed} chunk {chunk}")
+        for b, out in zip(branches, outs):
+            q, k, v = (dev_tensor(torch, b.cfg, 0, chunk, steps, t, Lq) for t in "qkv")
+            b.h.chunk_attention(0, q, k, v, out, cfg.C, f0, True)
+            b.oracles[0].write_chunk(host_bits(b.cfg, 0, chunk, steps, "k", Lq), host_bits(b.cfg, 0, chunk, steps, "v", Lq),
+                                     cfg.C, f0)
+            b.f0[0] = f0 + cfg.C
+    torch.cuda.synchronize()
+    for b in branches:
+        b.check_cache(0)
+        assert b.h.poll_device_status() == rkv.OK
+        b.h.close()
