@@ -201,6 +201,55 @@ def _cross_with_positions():
     return cross_attention
 
 
+def _chunk_attention_rotating_v():
+    """The layer's attention with V rotated by the keys' positions, like K."""
+    def chunk_attention(self, q_bits, k_bits, v_bits, n_frames, start_frame, commit, rows=None, heads=None,
+                        rope_out_bf16=False):
+        self._check_order(start_frame)
+        chunk = self._split_frames(k_bits, v_bits, n_frames, start_frame)
+        window = self.cache.after_append(chunk)
+        hs = list(range(self.H)) if heads is None else list(heads)
+        k = np.concatenate([f.k for f in window], axis=0)[:, hs, :]
+        v = np.concatenate([f.v for f in window], axis=0)[:, hs, :]
+        if self.rope_mode == self.RELATIVE_SLOTS:
+            k_ids = rope.time_ids_slot_order(len(window))
+            q_ids = k_ids[len(window) - n_frames:]
+        else:
+            k_ids = self.time_ids([f.frame for f in window], start_frame, n_frames)
+            q_ids = self.time_ids([start_frame + i for i in range(n_frames)], start_frame, n_frames)
+        k_pos = rope.token_positions(k_ids, self.T, self.grid_w)
+        k_rot = rope.rotate(bf16.to_f64(k), k_pos, self.theta, self.pairs)
+        v_rot = rope.rotate(bf16.to_f64(v), k_pos, self.theta, self.pairs)
+        q = np.asarray(q_bits, dtype=np.uint16).reshape(n_frames * self.T, self.H, self.d)[:, hs, :]
+        q_pos = rope.token_positions(q_ids, self.T, self.grid_w)
+        if rows is not None:
+            q, q_pos = q[np.asarray(rows)], q_pos[np.asarray(rows)]
+        out = attention.attend(rope.rotate(bf16.to_f64(q), q_pos, self.theta, self.pairs), k_rot, v_rot)
+        if commit:
+            self.cache.slots = window
+            self.committed += n_frames
+        return out
+    return chunk_attention
+
+
+def _chunk_attention_ignoring_rope_out_bf16():
+    orig = layer.OracleLayer.chunk_attention
+
+    def chunk_attention(self, q_bits, k_bits, v_bits, n_frames, start_frame, commit, rows=None, heads=None,
+                        rope_out_bf16=False):
+        return orig(self, q_bits, k_bits, v_bits, n_frames, start_frame, commit, rows, heads)
+    return chunk_attention
+
+
+def _slot_query_ids_from_window_start():
+    orig = rope.time_ids_slot_order
+
+    def time_ids_slot_order(n_visible):
+        ids = orig(n_visible)
+        return ids[::-1].copy()     # ids counted from the other end of the window
+    return time_ids_slot_order
+
+
 # ------------------------------------------------------------------ flow
 def _x0_renoise_with(kind):
     def x0_renoise_f64(xt, v, eps, sigma, sigma_next):
@@ -224,8 +273,22 @@ def _cfg_with(kind):
         u = np.asarray(v_uncond, dtype=np.float64)
         if kind == "swapped":
             return c + scale * (u - c)
+        if kind == "scale_on_u":
+            return scale * u + (c - u)
         return scale * (c - u)
     return cfg_combine_f64
+
+
+def _x0_renoise_sigma_for_next():
+    def x0_renoise_f64(xt, v, eps, sigma, sigma_next):
+        xt = np.asarray(xt, dtype=np.float64)
+        v = np.asarray(v, dtype=np.float64)
+        x0 = xt - sigma * v
+        if sigma_next < 0:
+            return x0, None
+        eps = np.asarray(eps, dtype=np.float64)
+        return x0, (1.0 - sigma) * x0 + sigma * eps     # renoised to the current sigma
+    return x0_renoise_f64
 
 
 # ------------------------------------------------------------------ bf16
@@ -299,6 +362,12 @@ MUTANTS = {
     "flow_renoise_from_xt": lambda: _rebind([(flow, "x0_renoise_f64")], _x0_renoise_with("renoise_from_xt")),
     "cfg_branches_swapped": lambda: _rebind([(flow, "cfg_combine_f64")], _cfg_with("swapped")),
     "cfg_missing_base": lambda: _rebind([(flow, "cfg_combine_f64")], _cfg_with("no_base")),
+    "cfg_scale_on_u": lambda: _rebind([(flow, "cfg_combine_f64")], _cfg_with("scale_on_u")),
+    "flow_renoise_to_current_sigma": lambda: _rebind([(flow, "x0_renoise_f64")], _x0_renoise_sigma_for_next()),
+    "layer_values_rotated_like_keys": lambda: setattr(layer.OracleLayer, "chunk_attention", _chunk_attention_rotating_v()),
+    "layer_ignores_rope_out_bf16": lambda: setattr(layer.OracleLayer, "chunk_attention",
+                                                   _chunk_attention_ignoring_rope_out_bf16()),
+    "rope_slot_ids_reversed": lambda: _rebind([(rope, "time_ids_slot_order")], _slot_query_ids_from_window_start()),
     # bf16
     "bf16_truncates": lambda: _patch_from_f64(_from_f64_with("truncate")),
     "bf16_ties_away": lambda: _patch_from_f64(_from_f64_with("ties_away")),
