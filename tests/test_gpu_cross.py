@@ -135,3 +135,26 @@ def test_cross_errors_launch_nothing():
     torch.cuda.synchronize()
     assert bool((out == 0).all())
     h.close()
+
+
+def test_cross_longest_text_context():
+    """The largest text context the library takes (65536 tokens, 512 key tiles in one
+    segment) element by element against the oracle, with a ragged query count; one more
+    token is refused before anything is launched."""
+    H, n_text, n_q = 1, 65536, 300
+    h = rkv.RollingKV(1, H, 128, 4, 6, 2, OracleLayer.ABSOLUTE)
+    kt, ktb = _pair(H, n_text, synth.stream_key(0, 74, 1))
+    vt, vtb = _pair(H, n_text, synth.stream_key(0, 74, 2))
+    h.set_text_kv(0, kt, vt)
+    orc = _oracle(H)
+    orc.set_text_kv(ktb, vtb)
+    q, qb = _pair(H, n_q, synth.stream_key(0, 75))
+    out = torch.empty_like(q)
+    h.cross_attention(0, q, out)
+    torch.cuda.synchronize()
+    assert_close(to_bits(out), orc.cross_attention(qb), "cross n_text 65536")
+    k2 = torch.zeros((n_text + 1, H, 128), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(rkv.RkvError):
+        h.set_text_kv(0, k2, k2)
+    assert h.poll_device_status() == rkv.OK
+    h.close()
