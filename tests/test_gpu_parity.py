@@ -79,6 +79,31 @@ def test_rope_apply_within_one_ulp(mode):
     h.close()
 
 
+def test_rope_apply_top_of_time_table():
+    """Absolute ids at the top of the library's time table (65534, 65535: angles of tens of
+    thousands of radians, the (cos, sin) rows built in fp64 on the host) within one bf16 ulp
+    of the oracle; a chunk reaching id 65536 is refused before anything is launched."""
+    H, gh, gw, W = 2, 4, 5, 6
+    T = gh * gw
+    h = rkv.RollingKV(1, H, 128, T, W, 2, ABS)
+    h.set_rope_grid(gh, gw)
+    orc = OracleLayer(H, 128, T, gh, gw, W, 2, ABS)
+    x = _dev_bits(synth.stream_key(1, 65534), 2 * T * H * 128).view(2 * T, H, 128)
+    xb = to_bits(x)
+    h.rope_apply(x, 2, 65534, 0)
+    torch.cuda.synchronize()
+    ref = orc.rope_apply(xb, 2, 65534)
+    after = to_bits(x)
+    got = bf16.to_f64(after)
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref), 2.0 ** -126))) - 7)
+    assert np.all(np.abs(got - ref) <= ulp)
+    with pytest.raises(rkv.RkvError):
+        h.rope_apply(x, 2, 65535, 0)
+    torch.cuda.synchronize()
+    assert np.array_equal(to_bits(x), after)   # the refused call launched nothing
+    h.close()
+
+
 SMALL = [
     Config("tiny-abs", 1, H=2, grid_h=4, grid_w=4, C=2, W=6, S=2, rope_mode=ABS, chunks=10),
     Config("tiny-rel-refs", 2, H=2, grid_h=4, grid_w=4, C=2, W=6, S=2, rope_mode=REL, refs=2, chunks=10),
