@@ -188,6 +188,55 @@ def test_outputs_are_deterministic():
     h.close()
 
 
+def test_two_handles_on_two_streams_match_sequential():
+    """Handles share no device state: two handles driven concurrently on two streams (reads
+    and commits interleaved, no ordering between the streams) give bit for bit the outputs
+    and caches of the same calls run one after another on one stream."""
+    cfgs = [Config("conc-a", 30, H=2, grid_h=8, grid_w=10, C=3, W=7, S=2, rope_mode=REL, chunks=5, reads=2),
+            Config("conc-b", 31, H=3, grid_h=10, grid_w=20, C=2, W=5, S=1, rope_mode=ABS, chunks=5, reads=2)]
+
+    def run(streams):
+        hs, outs = [], []
+        for c in cfgs:
+            h = rkv.RollingKV(1, c.H, 128, c.T, c.W, c.S, c.rope_mode)
+            h.set_rope_grid(c.grid_h, c.grid_w)
+            hs.append(h)
+        inputs = [[[[dev_tensor(torch, c, 0, chunk, call, t, c.Lq) for t in ("q", "k", "v")]
+                    for call in range(c.reads + 1)] for chunk in range(c.chunks)] for c in cfgs]
+        res = [[torch.empty((c.Lq, c.H, 128), dtype=torch.bfloat16, device="cuda")
+                for _ in range(c.chunks * (c.reads + 1))] for c in cfgs]
+        torch.cuda.synchronize()
+        for chunk in range(5):
+            for i, (c, h) in enumerate(zip(cfgs, hs)):
+                st = streams[i]
+                with torch.cuda.stream(st):
+                    for call in range(c.reads + 1):
+                        q, k, v = inputs[i][chunk][call]
+                        h.chunk_attention(0, q, k, v, res[i][chunk * (c.reads + 1) + call], c.C, chunk * c.C,
+                                          call == c.reads, stream=st.cuda_stream)
+        torch.cuda.synchronize()
+        for i, (c, h) in enumerate(zip(cfgs, hs)):
+            outs.append([to_bits(o) for o in res[i]] + [to_bits(_cache_view(h, c, w)) for w in (0, 1)])
+            assert h.poll_device_status() == rkv.OK
+            h.close()
+        return outs
+
+    one = torch.cuda.Stream()
+    seq = run([one, one])
+    par = run([torch.cuda.Stream(), torch.cuda.Stream()])
+    for a, b in zip(seq, par):
+        assert len(a) == len(b) and all(np.array_equal(x, y) for x, y in zip(a, b))
+
+
+def _cache_view(h, c, which):
+    ptr = h.cache_ptrs(0)[which]
+    n = c.H * c.W * c.T * 128
+
+    class _A:
+        __cuda_array_interface__ = {"shape": (n,), "typestr": "<i2", "data": (ptr, False), "version": 3}
+    return torch.as_tensor(_A(), device="cuda").view(torch.bfloat16)
+
+
 @pytest.mark.parametrize("sink_score", [-2000.0, -150.0, 400.0])
 @pytest.mark.parametrize("mode", [ABS, REL])
 def test_score_jumps_between_key_tiles(sink_score, mode):
