@@ -378,7 +378,9 @@ def run_rkv(args):
                      "traffic_source": traffic_src,
                      "kernel": "chunk_attention_kernel", "peak_source": f"{pk_kind} bf16_tflops_sustained",
                      "frac_of_burst": (achieved / pk["bf16_tflops"]) if achieved else None,
-                     "mean_kernel_ms": mean_kernel_ms, "launches_timed": len(kernel_ms),
+                     "mean_kernel_ms": mean_kernel_ms,
+                     "median_kernel_ms": statistics.median(kernel_ms) if kernel_ms else None,
+                     "launches_timed": len(kernel_ms),
                      "flops_per_launch": flops / max(1, 5 * n_layers * args.steps)},
         "frames_per_s_per_layer": C * n_layers * args.steps * world / (ms / 1e3),
         "rollout": rollout,
