@@ -71,6 +71,32 @@ def test_planner_matches_oracle_cache(W, S, C, refs):
         committed += C
 
 
+def test_planner_matches_oracle_cache_mixed_chunk_sizes():
+    """Random windows and random sequences of chunk sizes (every size the window takes), the
+    plan of each chunk against the oracle's literal cache (hypothesis, derandomized)."""
+    hypothesis = pytest.importorskip("hypothesis")
+    st = hypothesis.strategies
+
+    @hypothesis.settings(max_examples=300, deadline=None, derandomize=True)
+    @hypothesis.given(st.integers(1, 40).flatmap(
+        lambda W: st.tuples(st.just(W), st.integers(0, W - 1)).flatmap(
+            lambda ws: st.tuples(st.just(ws[0]), st.just(ws[1]),
+                                 st.lists(st.integers(1, ws[0] - ws[1]), min_size=1, max_size=40)))))
+    def check(args):
+        W, S, sizes = args
+        cache = RollingCache(W, S)
+        committed = 0
+        for C in sizes:
+            segs = rkv.plan_window(W, S, committed, C, committed)
+            assert 1 <= len(segs) <= 4
+            assert segs[-1][0] == 1 and segs[-1][2] == C and segs[-1][3] == committed
+            assert _frames_from_plan(segs, W, S) == cache.after_append(list(range(committed, committed + C)))
+            cache.append(list(range(committed, committed + C)))
+            committed += C
+
+    check()
+
+
 def test_planner_errors():
     with pytest.raises(rkv.RkvError) as e:
         rkv.plan_window(6, 2, 4, 2, 3)
