@@ -15,7 +15,7 @@ import pytest
 import synth
 from oracle import bf16, flow as oflow
 from oracle.layer import OracleLayer
-from rollout import Config, Rollout, assert_close, dev_tensor, host_bits, to_bits
+from rollout import Config, Rollout, assert_close, cache_logical_bits, dev_tensor, host_bits, to_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -185,6 +185,41 @@ def test_outputs_are_deterministic():
         h.chunk_attention(0, q, k, v, o, cfg.C, 0, False)
         outs.append(to_bits(o))
     assert np.array_equal(outs[0], outs[1]) and np.array_equal(outs[0], outs[2])
+    h.close()
+
+
+@pytest.mark.parametrize("mode", [ABS, REL, SLOTS])
+def test_mixed_chunk_sizes(mode):
+    """Chunks of 1 to 4 frames in an irregular order after two reference frames, through
+    eviction and ring wrap: every read and commit element by element, the cache bit for bit
+    after every commit."""
+    H, gh, gw, W, S = 2, 4, 5, 9, 2
+    T = gh * gw
+    sizes = [1, 3, 2, 4, 1, 1, 3, 2, 4, 2, 1, 3, 4, 1, 2]
+    h = rkv.RollingKV(1, H, 128, T, W, S, mode)
+    h.set_rope_grid(gh, gw)
+    orc = OracleLayer(H, 128, T, gh, gw, W, S, mode)
+    cfg = Config("mixed", 40 + mode, H=H, grid_h=gh, grid_w=gw, C=1, W=W, S=S, rope_mode=mode)
+    kr, vr = (dev_tensor(torch, cfg, 0, -1, 0, t, S * T) for t in ("k", "v"))
+    h.write_chunk(0, kr, vr, S, 0)
+    orc.write_chunk(host_bits(cfg, 0, -1, 0, "k", S * T), host_bits(cfg, 0, -1, 0, "v", S * T), S, 0)
+    f0 = S
+    for i, C in enumerate(sizes):
+        n = C * T
+        for call in range(2):
+            commit = call == 1
+            q, k, v = (dev_tensor(torch, cfg, 0, i, call, t, n) for t in ("q", "k", "v"))
+            out = torch.empty((n, H, 128), dtype=torch.bfloat16, device="cuda")
+            h.chunk_attention(0, q, k, v, out, C, f0, commit)
+            ref = orc.chunk_attention(*(host_bits(cfg, 0, i, call, t, n) for t in ("q", "k", "v")), C, f0, commit)
+            torch.cuda.synchronize()
+            assert_close(to_bits(out), ref, f"mixed mode {mode} chunk {i} (C={C}) call {call}")
+        f0 += C
+        frames, kb, vb = cache_logical_bits(h, torch, cfg, 0)
+        assert frames == orc.logical_frames()
+        ok_, ov = orc.logical_kv_bits()
+        assert np.array_equal(kb, ok_) and np.array_equal(vb, ov)
+    assert h.poll_device_status() == rkv.OK
     h.close()
 
 
