@@ -223,6 +223,43 @@ def test_mixed_chunk_sizes(mode):
     h.close()
 
 
+@pytest.mark.parametrize("mode", [ABS, REL])
+def test_reset_replays_bit_for_bit(mode):
+    """rkv_reset returns a handle to its just-created state: the same rollout (reference
+    frames, then reads and commits through eviction and wrap) run again after a reset gives
+    bit for bit the same outputs, slot map and cache bytes; in relative mode this includes
+    the rotated ring, whose validity is keyed on the chunk's position."""
+    cfg = Config("reset", 45 + mode, H=2, grid_h=4, grid_w=5, C=2, W=6, S=2, rope_mode=mode, refs=1, chunks=7,
+                 reads=2)
+    h = rkv.RollingKV(1, cfg.H, 128, cfg.T, cfg.W, cfg.S, mode)
+    h.set_rope_grid(cfg.grid_h, cfg.grid_w)
+
+    def rollout():
+        outs = []
+        kr, vr = (dev_tensor(torch, cfg, 0, -1, 0, t, cfg.refs * cfg.T) for t in ("k", "v"))
+        h.write_chunk(0, kr, vr, cfg.refs, 0)
+        f0 = cfg.refs
+        for chunk in range(cfg.chunks):
+            for call in range(cfg.reads + 1):
+                q, k, v = (dev_tensor(torch, cfg, 0, chunk, call, t, cfg.Lq) for t in ("q", "k", "v"))
+                out = torch.empty((cfg.Lq, cfg.H, 128), dtype=torch.bfloat16, device="cuda")
+                h.chunk_attention(0, q, k, v, out, cfg.C, f0, call == cfg.reads)
+                outs.append(to_bits(out))
+            f0 += cfg.C
+        frames, kb, vb = cache_logical_bits(h, torch, cfg, 0)
+        return outs, list(h.slot_frames(0)), frames, kb, vb
+
+    first = rollout()
+    h.reset()
+    assert h.frames_committed(0) == 0 and all(f < 0 for f in h.slot_frames(0))
+    second = rollout()
+    assert len(first[0]) == len(second[0]) and all(np.array_equal(a, b) for a, b in zip(first[0], second[0]))
+    assert first[1] == second[1] and first[2] == second[2]
+    assert np.array_equal(first[3], second[3]) and np.array_equal(first[4], second[4])
+    assert h.poll_device_status() == rkv.OK
+    h.close()
+
+
 def test_two_handles_on_two_streams_match_sequential():
     """Handles share no device state: two handles driven concurrently on two streams (reads
     and commits interleaved, no ordering between the streams) give bit for bit the outputs
