@@ -191,8 +191,10 @@ def test_outputs_are_deterministic():
 @pytest.mark.parametrize("mode", [ABS, REL, SLOTS])
 def test_mixed_chunk_sizes(mode):
     """Chunks of 1 to 4 frames in an irregular order after two reference frames, through
-    eviction and ring wrap: every read and commit element by element, the cache bit for bit
-    after every commit."""
+    eviction and ring wrap, with one group of frames written mid-rollout without attention
+    (rkv_write_chunk: in absolute mode its rotated keys come from the caller's k, not from a
+    call's rotated chunk): every read and commit element by element, the cache bit for bit
+    after every chunk."""
     H, gh, gw, W, S = 2, 4, 5, 9, 2
     T = gh * gw
     sizes = [1, 3, 2, 4, 1, 1, 3, 2, 4, 2, 1, 3, 4, 1, 2]
@@ -206,6 +208,12 @@ def test_mixed_chunk_sizes(mode):
     f0 = S
     for i, C in enumerate(sizes):
         n = C * T
+        if i == 6:   # frames kept without attention, mid-rollout
+            kw, vw = (dev_tensor(torch, cfg, 0, i, 9, t, n) for t in ("k", "v"))
+            h.write_chunk(0, kw, vw, C, f0)
+            orc.write_chunk(host_bits(cfg, 0, i, 9, "k", n), host_bits(cfg, 0, i, 9, "v", n), C, f0)
+            f0 += C
+            continue
         for call in range(2):
             commit = call == 1
             q, k, v = (dev_tensor(torch, cfg, 0, i, call, t, n) for t in ("q", "k", "v"))
