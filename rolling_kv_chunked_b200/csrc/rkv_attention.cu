@@ -42,6 +42,7 @@
 // kStatusTimeout in the status word, stops issuing work, waits (bounded) for the
 // copies and MMAs it already issued, frees TMEM and returns.
 #include <cfloat>
+#include <mutex>
 
 #include "numeric.cuh"
 #include "ptx_sm100.cuh"
@@ -573,14 +574,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 cudaError_t launch_attention(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_vc,
                              const CUtensorMap& tm_vn, const AttnParams& p, cudaStream_t stream) {
-  static int configured_device = -1;
+  // the dynamic shared-memory limit is a per-device setting: raised once on every device
+  // this process launches on, whichever host thread gets there first
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static bool configured[kMaxDevices] = {};
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
-  if (configured_device != dev) {
-    err = cudaFuncSetAttribute(chunk_attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (err != cudaSuccess) return err;
-    configured_device = dev;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!configured[dev]) {
+      err = cudaFuncSetAttribute(chunk_attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+      if (err != cudaSuccess) return err;
+      configured[dev] = true;
+    }
   }
   dim3 grid((p.Lq + 2 * kBM - 1) / (2 * kBM), p.H);
   chunk_attention_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_q, tm_k, tm_vc, tm_vn, p);
