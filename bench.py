@@ -12,7 +12,11 @@ to steady state (full window, evictions firing) before warm-up.
 Metric: query tokens / s per layer (5 * Lq per layer per step), whole job over all ranks.
 Multi-GPU: independent replicas (one layer each), no data-path collective.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config abot|480p|720p|long|abot_cfg] [--impl rkv|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 720p|480p|abot|long|abot_cfg] [--impl rkv|reference]
+
+The default workload is the 720p one (the largest that fits one GPU); the line also carries
+compact records of the ABot and 480P workloads (``workloads``). ``--gpus N`` outside a
+launcher starts N ranks under torch.distributed.run itself.
 
 ``--config abot_cfg`` measures the guided (classifier-free guidance) mode instead: two caches,
 40 guided steps per chunk with the guidance combine fused into the unconditional read.
@@ -206,7 +210,56 @@ def visible_keys(cfg, committed, f0):
     return sum(n for _, _, n, _ in rkv.plan_window(cfg["W"], cfg["S"], committed, cfg["C"], f0)) * T
 
 
+# a timed region at least this long is compared with the sustained (power-capped) bf16 peak;
+# a shorter one with the burst peak
+SUSTAINED_REGION_S = 1.0
+# the workloads reported beside the headline one, each as a compact record
+SIDE_WORKLOADS = ("abot", "480p")
+
+
+def config_record(cfg, world):
+    """The `config` of the bench line: the workload and its sizes (both arms print the same)."""
+    T = cfg["gh"] * cfg["gw"]
+    Lq = cfg["C"] * T
+    n_layers = cfg.get("layers", 1)
+    return {"workload": cfg["workload"], "queries_per_call": Lq, "keys_per_call": cfg["W"] * T,
+            "calls_per_step": 5 * n_layers, "layers": n_layers,
+            "parallelism": f"replicas x{world} (no data-path collective)",
+            "l2": f"inputs larger than L2 ({19 * Lq * cfg['H'] * 128 * 2 / 1e6:.0f} MB per step)"}
+
+
+def peak_for_region(pk, region_s):
+    """(peak TFLOP/s, which one) for a timed region of region_s seconds."""
+    if region_s >= SUSTAINED_REGION_S:
+        return pk["bf16_tflops_sustained"], "bf16_tflops_sustained"
+    return pk["bf16_tflops"], "bf16_tflops"
+
+
 def run_rkv(args):
+    import torch
+    import torch.distributed as dist
+
+    world, rank, local = rank_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
+    result = measure_workload(args, args.config, headline=True)
+    if CONFIGS[args.config].get("layers", 1) == 1 and not args.no_side:
+        result["workloads"] = {}
+        for name in SIDE_WORKLOADS:
+            if name != args.config:
+                result["workloads"][name] = measure_workload(args, name, headline=False)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+def measure_workload(args, name, headline):
+    """One workload: the timed steps (inputs resident in HBM), and for the headline also the
+    whole rollout, the end-to-end pass from host buffers, the HBM-bound kernels, the
+    cross-attention and the CPU baseline; side workloads give a compact record."""
     import torch
     import torch.distributed as dist
 
@@ -214,12 +267,7 @@ def run_rkv(args):
     import synth
 
     world, rank, local = rank_env()
-    torch.cuda.set_device(local)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
-
-    cfg = CONFIGS[args.config]
+    cfg = CONFIGS[name]
     H, C, W, S = cfg["H"], cfg["C"], cfg["W"], cfg["S"]
     T = cfg["gh"] * cfg["gw"]
     Lq = C * T
@@ -327,6 +375,29 @@ def run_rkv(args):
     tokens = 5 * n_layers * Lq * args.steps * world
     value = tokens / (ms / 1e3)
 
+    pk, pk_kind = peaks()
+    mean_kernel_ms = sum(kernel_ms) / max(1, len(kernel_ms))
+    achieved = flops / (sum(kernel_ms) / 1e3) / 1e12 if kernel_ms else None
+    region_s = ms / 1e3
+    peak, peak_name = peak_for_region(pk, region_s)
+    n_launch = 5 * n_layers * args.steps
+    attn = {"achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": (achieved / peak) if achieved else None,
+            "peak_source": f"{pk_kind} {peak_name} (timed region {region_s:.2f} s; sustained peak from "
+                           f"{SUSTAINED_REGION_S:g} s up)",
+            "frac_of_burst": (achieved / pk["bf16_tflops"]) if achieved else None,
+            "frac_of_sustained": (achieved / pk["bf16_tflops_sustained"]) if achieved else None,
+            "mean_kernel_ms": mean_kernel_ms,
+            "median_kernel_ms": statistics.median(kernel_ms) if kernel_ms else None,
+            "launches_timed": len(kernel_ms), "flops_per_launch": flops / max(1, n_launch)}
+    if not headline:
+        hbm = None if args.no_hbm else measure_hbm_kernels(torch, rkv, synth, cfg, rank)
+        h.close()
+        del pool, outs, x0, xn
+        torch.cuda.empty_cache()
+        return {"workload": cfg["workload"], "value": value, "unit": UNIT, "steps": args.steps,
+                "ms_per_step": ms / args.steps, "queries_per_call": Lq, "keys_per_call": W * T,
+                "attention": attn, "hbm_kernels": hbm, "clocks": clk}
+
     # ---- a whole rollout from an empty cache: the reference frames, then every chunk of the
     # workload's video (4 reads + 1 commit each), warm-up chunks with short windows included
     rollout = None
@@ -360,28 +431,14 @@ def run_rkv(args):
     hbm = None if args.no_hbm or n_layers > 1 else measure_hbm_kernels(torch, rkv, synth, cfg, rank)
     cross = None if args.no_hbm or n_layers > 1 else measure_cross_attention(torch, rkv, synth, cfg, rank)
 
-    pk, pk_kind = peaks()
-    traffic, traffic_src = profiled_traffic(args.config)
-    mean_kernel_ms = sum(kernel_ms) / max(1, len(kernel_ms))
-    achieved = flops / (sum(kernel_ms) / 1e3) / 1e12 if kernel_ms else None
-    peak = pk["bf16_tflops_sustained"]
+    traffic, traffic_src = profiled_traffic(name)
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": cfg["workload"], "queries_per_call": Lq, "keys_per_call": W * T,
-                   "calls_per_step": 5 * n_layers, "layers": n_layers,
-                   "parallelism": f"replicas x{world} (no data-path collective)",
-                   "l2": f"inputs larger than L2 ({(15 * Lq * H * 128 + 4 * Lq * H * 128) * 2 / 1e6:.0f} MB per step)"},
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": (achieved / peak) if achieved else None, "traffic": traffic,
-                     "traffic_source": traffic_src,
-                     "kernel": "chunk_attention_kernel", "peak_source": f"{pk_kind} bf16_tflops_sustained",
-                     "frac_of_burst": (achieved / pk["bf16_tflops"]) if achieved else None,
-                     "mean_kernel_ms": mean_kernel_ms,
-                     "median_kernel_ms": statistics.median(kernel_ms) if kernel_ms else None,
-                     "launches_timed": len(kernel_ms),
-                     "flops_per_launch": flops / max(1, 5 * n_layers * args.steps)},
+        "config": config_record(cfg, world),
+        "roofline": {"bound": "tensor", **attn, "traffic": traffic, "traffic_source": traffic_src,
+                     "kernel": "chunk_attention_kernel"},
         "frames_per_s_per_layer": C * n_layers * args.steps * world / (ms / 1e3),
         "rollout": rollout,
         "e2e": e2e,
@@ -393,10 +450,9 @@ def run_rkv(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(cfg, budget_s=args.cpu_seconds)
     h.close()
-    if world > 1:
-        dist.destroy_process_group()
-    if rank == 0:
-        print(json.dumps(result), flush=True)
+    del pool, outs, x0, xn
+    torch.cuda.empty_cache()
+    return result
 
 
 def run_cfg(args):
@@ -754,20 +810,33 @@ def cpu_threads():
         return os.cpu_count()
 
 
-def cpu_baseline(cfg, budget_s=10.0, heads=2):
-    """The oracle as it stands, on a bounded sample: `heads` of H heads of steady-state
-    denoise reads (all queries, full window), repeated for ~budget_s, scaled by H / heads."""
+# the oracle's sample of one call: this many query rows (evenly spaced over the chunk) of one
+# head against the full steady-state window, scaled to all rows and heads
+SAMPLE_ROWS = 1024
+
+
+def _sample_rows(Lq):
+    import numpy as np
+    n = min(SAMPLE_ROWS, Lq)
+    return np.unique(np.linspace(0, Lq - 1, n).round().astype(np.int64))
+
+
+def cpu_baseline(cfg, budget_s=10.0):
+    """The oracle as it stands, on a bounded sample: steady-state denoise reads of one head,
+    SAMPLE_ROWS query rows against the full window, repeated for ~budget_s, scaled by
+    H * Lq / rows."""
     orc, q, f0 = _oracle_steady_layer(cfg)
     C, H = cfg["C"], cfg["H"]
     T = cfg["gh"] * cfg["gw"]
+    rows = _sample_rows(C * T)
     n, t0 = 0, time.perf_counter()
     while True:
-        orc.chunk_attention(q, q, q, C, f0, False, heads=list(range(heads)))
+        orc.chunk_attention(q, q, q, C, f0, False, heads=[0], rows=rows)
         n += 1
         el = time.perf_counter() - t0
         if el >= budget_s:
             break
-    per_call_s = el / n * (H / heads)
+    per_call_s = el / n * H * (C * T) / len(rows)
     # the oracle's x0 / renoise step (K4) on an eighth of the workload's latent
     from oracle import flow as oflow
     import synth
@@ -777,8 +846,8 @@ def cpu_baseline(cfg, budget_s=10.0, heads=2):
     oflow.x0_renoise_bf16(xt, v, eps, 1.0, 0.75)
     flow_s = time.perf_counter() - t1
     return {"value": C * T / per_call_s, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-            "sample": f"{n} steady-state reads x {heads} of {H} heads (all {C * T} queries vs {cfg['W'] * T} keys), "
-                      f"numpy fp64, scaled by {H}/{heads}",
+            "sample": f"{n} steady-state reads of 1 of {H} heads, {len(rows)} of {C * T} query rows vs "
+                      f"{cfg['W'] * T} keys, numpy fp64, scaled by {H} x {C * T}/{len(rows)}",
             "flow_x0_renoise": {"GB/s": 10 * n_el / flow_s / 1e9, "elements": n_el,
                                 "sample": "one call on an eighth of the latent, sigma 1.0 -> 0.75, numpy fp64"}}
 
@@ -792,22 +861,22 @@ def run_reference(args):
     C, H = cfg["C"], cfg["H"]
     T = cfg["gh"] * cfg["gw"]
     Lq = C * T
-    heads = [0]
+    rows = _sample_rows(Lq)
     for _ in range(args.warmup):
-        orc.chunk_attention(q, q, q, C, f0, False, heads=heads)
+        orc.chunk_attention(q, q, q, C, f0, False, heads=[0], rows=rows)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        orc.chunk_attention(q, q, q, C, f0, False, heads=heads)
+        orc.chunk_attention(q, q, q, C, f0, False, heads=[0], rows=rows)
     el = time.perf_counter() - t0
-    per_call_s = el / args.steps * H
+    per_call_s = el / args.steps * H * Lq / len(rows)
     value = Lq / per_call_s
-    sample = (f"each step: one steady-state read, 1 of {H} heads (all {Lq} queries vs {cfg['W'] * T} keys), "
-              f"scaled by {H}")
+    sample = (f"each step: one steady-state read of 1 of {H} heads, {len(rows)} of {Lq} query rows vs "
+              f"{cfg['W'] * T} keys, scaled by {H} x {Lq}/{len(rows)}")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": cfg["workload"]},
+        "data": "synthetic", "config": config_record(cfg, world),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
@@ -815,7 +884,8 @@ def run_reference(args):
 
 def run_isolated(args):
     """A few launches of one kernel at the workload's sizes and nothing else, for profiler
-    captures (``ncu -k <kernel> -s 1 -c 1 python bench.py --isolate ...``): ``commit``
+    captures (``ncu -k <kernel> -s 1 -c 1 python bench.py --isolate ...``): ``attention``
+    (steady-state reads, see run_isolated_attention), ``commit``
     (rkv_write_chunk: the ring write-back), ``rope`` (rkv_rope_apply of one chunk's
     [Lq, H, 128] tensor), ``flow`` (rkv_flow_x0_renoise on the [Lq, H*128] latent, renoise
     on) or ``cross`` (rkv_cross_attention of the chunk's queries over 512 text tokens).
@@ -837,6 +907,9 @@ def run_isolated(args):
         synth.fill_normal_bf16_cuda(t.data_ptr(), t.numel(), synth.stream_key(0, 91, *f), 0, sp)
         return t
 
+    if args.isolate == "attention":
+        run_isolated_attention(args, torch, rkv, synth, cfg)
+        return
     per_set = {"commit": 2, "rope": 1, "flow": 5, "cross": 2}[args.isolate]
     n_sets = max(2, -(-int(256e6) // (per_set * n * 2)))
     sets = [[fill(torch.empty((Lq, H, 128), **bf), i, j) for j in range(per_set)] for i in range(n_sets)]
@@ -884,12 +957,87 @@ def run_isolated(args):
                       "us_per_launch": us, **work}), flush=True)
 
 
+def run_isolated_attention(args, torch, rkv, synth, cfg):
+    """Steady-state attention reads of the workload and as little else as possible: the window
+    is filled by rkv_write_chunk (two launches: the sinks, then the rest), then --reps denoise
+    reads of the next chunk run (each the RoPE pre-pass plus one attention launch). Holds the
+    layer's caches and one q / k / v set (~3.5 GB at 720p), for profiler captures
+    (``ncu -k regex:chunk_attention -c 1``)."""
+    H, C, W, S = cfg["H"], cfg["C"], cfg["W"], cfg["S"]
+    T = cfg["gh"] * cfg["gw"]
+    Lq = C * T
+    st = torch.cuda.current_stream()
+    sp = st.cuda_stream
+    bf = dict(dtype=torch.bfloat16, device="cuda")
+    h = rkv.RollingKV(1, H, 128, T, W, S, cfg["mode"])
+    h.set_rope_grid(cfg["gh"], cfg["gw"])
+    f = 0
+    for n in (S, W - S):
+        k = torch.empty((n * T, H, 128), **bf)
+        v = torch.empty((n * T, H, 128), **bf)
+        synth.fill_normal_bf16_cuda(k.data_ptr(), k.numel(), synth.stream_key(0, 92, f, 2), 0, sp)
+        synth.fill_normal_bf16_cuda(v.data_ptr(), v.numel(), synth.stream_key(0, 92, f, 3), 0, sp)
+        h.write_chunk(0, k, v, n, f, stream=sp)
+        f += n
+        del k, v
+    qkv = []
+    for tag in (1, 2, 3):
+        t = torch.empty((Lq, H, 128), **bf)
+        synth.fill_normal_bf16_cuda(t.data_ptr(), t.numel(), synth.stream_key(0, 92, f, tag), 0, sp)
+        qkv.append(t)
+    out = torch.empty((Lq, H, 128), **bf)
+    keys = visible_keys(cfg, f, f)
+    torch.cuda.synchronize()
+    h.timing_begin(args.reps)
+    for _ in range(args.reps):
+        h.chunk_attention(0, *qkv, out, C, f, False, stream=sp)
+    ms = h.timing_end(args.reps)
+    if h.poll_device_status(sp) != rkv.OK:
+        raise RuntimeError("device wait expired")
+    h.close()
+    print(json.dumps({"isolate": "attention", "config": args.config, "launches": args.reps,
+                      "us_per_launch": [x * 1e3 for x in ms], "queries": Lq, "keys": keys,
+                      "flops_per_launch": 4.0 * H * 128 * Lq * keys,
+                      "algorithmic_bytes_per_launch": algorithmic_attention_bytes(cfg, keys, flow=False)}),
+          flush=True)
+
+
+def algorithmic_attention_bytes(cfg, keys, flow):
+    """Bytes one attention launch must move at least: Q, K and V of the visible window read
+    once per head, O written; with the fused x0 / renoise epilogue also xt and eps read and x0,
+    xt' written (four latent-sized streams)."""
+    H = cfg["H"]
+    Lq = cfg["C"] * cfg["gh"] * cfg["gw"]
+    b = 2 * 128 * H * (Lq + 2 * keys + Lq)
+    if flow:
+        b += 4 * 2 * 128 * H * Lq
+    return b
+
+
+def relaunch_ranks(n, impl):
+    """--gpus N without a launcher: start N ranks of this same command line under
+    torch.distributed.run (one process per GPU, rendezvous on 127.0.0.1) and return its exit
+    status. The GPU arm needs N visible GPUs; the reference arm runs on the host."""
+    if impl == "rkv":
+        import torch
+        have = torch.cuda.device_count()
+        if have < n:
+            raise SystemExit(f"--gpus {n}: only {have} CUDA device(s) visible")
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", str(n),
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", default="abot", choices=sorted(CONFIGS) + sorted(CFG_CONFIGS))
+    ap.add_argument("--config", default="720p", choices=sorted(CONFIGS) + sorted(CFG_CONFIGS))
     ap.add_argument("--impl", default="rkv", choices=["rkv", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -897,7 +1045,9 @@ def main():
     ap.add_argument("--no-hbm", action="store_true",
                     help="skip the side measurements (HBM-bound kernels, cross-attention)")
     ap.add_argument("--no-rollout", action="store_true", help="skip the whole-rollout pass")
-    ap.add_argument("--isolate", choices=["commit", "rope", "flow", "cross"],
+    ap.add_argument("--no-side", action="store_true",
+                    help="skip the compact records of the other single-layer workloads")
+    ap.add_argument("--isolate", choices=["attention", "commit", "rope", "flow", "cross"],
                     help="only launch this kernel --reps times at the config's sizes (for profiler captures)")
     ap.add_argument("--reps", type=int, default=3, help="launches of the --isolate kernel")
     args = ap.parse_args()
@@ -908,6 +1058,12 @@ def main():
         return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        sys.exit(relaunch_ranks(args.gpus, args.impl))
+    if int(os.environ.get("WORLD_SIZE", "1")) != args.gpus:
+        ap.error(f"--gpus {args.gpus} does not match the {os.environ.get('WORLD_SIZE', '1')} ranks launched")
     if args.impl == "reference":
         run_reference(args)
     elif args.config in CFG_CONFIGS:

@@ -263,17 +263,19 @@ int rkv_set_wait_limit(rkv_handle h, long long nanoseconds);
  *  n_window_frames frames the chunk attends to, in logical order (sinks,
  *  history, then the chunk's own n_frames frames last), token-major
  *  [n_window_frames*T, H, 128] bf16; frame_ids (host, n_window_frames ints) are
- *  their absolute frame indices, the last n_frames being start_frame.. .
- *  q and out are [n_frames*T, H, 128]. RoPE: theta 1e4, pairs 22/21/21, time id
- *  the frame index (RKV_ROPE_ABSOLUTE, ids < 4096) or re-based and clamped to
- *  [0, window_frames-1] (RKV_ROPE_RELATIVE). Output as rkv_chunk_attention.
+ *  their absolute frame indices, non-negative and strictly increasing, the last
+ *  n_frames being start_frame.. . q and out are [n_frames*T, H, 128]. RoPE: theta
+ *  1e4, pairs 22/21/21, time id the frame index (RKV_ROPE_ABSOLUTE, ids < 4096) or
+ *  re-based and clamped to [0, window_frames-1] (RKV_ROPE_RELATIVE; then
+ *  n_window_frames <= window_frames <= 4096). Output as rkv_chunk_attention.
  *  Scratch: one static device array of 32 MiB per device (RoPE tables, rotated
  *  Q and K, a status word), held from the library's first use on that device
  *  until exit. The first call on a device looks up the array's device address;
  *  make that first call before any stream capture. Calls share the array: calls
  *  that overlap on the GPU race. An expired device wait is not reported here.
- *  Errors: RKV_ERR_ARG, RKV_ERR_UNSUPPORTED (absolute id >= 4096, window in more
- *  than 7 runs of consecutive frames), RKV_ERR_CAPACITY (the window, queries and
+ *  Errors: RKV_ERR_ARG, RKV_ERR_UNSUPPORTED (absolute id >= 4096, relative
+ *  window_frames > 4096, window in more than 7 runs of consecutive frames),
+ *  RKV_ERR_CAPACITY (the window, queries and
  *  tables need more than the 32 MiB array), RKV_ERR_CUDA. Argument and size
  *  errors launch nothing.
  */

@@ -127,7 +127,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // 2^x for two lanes on the FMA / integer pipes instead of the special-function unit:
 // t = x + 1.5*2^23 rounds x to the nearest integer r (kept in t's low mantissa bits),
 // f = x - r in [-1/2, 1/2], 2^f by a degree-3 polynomial (max relative error 7.5e-5,
-// coefficients fitted for minimal relative error by rolling_kv_chunked_b200/exp2_poly.py),
+// coefficients fitted for minimal relative error by tests/exp2_poly.py),
 // then r is added to the exponent field (the bits of 1.5*2^23 vanish under << 23).
 // x is clamped to [-125, 126] so the result stays a positive normal number (a score far
 // above the reference then shows up as a huge tile sum, as it does on the other path).

@@ -111,28 +111,42 @@ extern "C" __attribute__((visibility("default"))) int rkv_chunk_attention_noallo
   using namespace rkv;
   if (!aligned16(q) || !aligned16(k_window) || !aligned16(v_window) || !aligned16(out) || frame_ids == nullptr)
     return RKV_ERR_ARG;
-  if (H <= 0 || tokens_per_frame <= 0 || grid_h <= 0 || grid_w <= 0 || grid_h * grid_w != tokens_per_frame ||
-      n_frames <= 0 || n_window_frames < n_frames || window_frames <= 0 || start_frame < 0)
+  if (H <= 0 || tokens_per_frame <= 0 || grid_h <= 0 || grid_w <= 0 ||
+      static_cast<long long>(grid_h) * grid_w != tokens_per_frame || n_frames <= 0 || n_window_frames < n_frames ||
+      window_frames <= 0 || start_frame < 0)
     return RKV_ERR_ARG;
   if (rope_mode != RKV_ROPE_ABSOLUTE && rope_mode != RKV_ROPE_RELATIVE) return RKV_ERR_ARG;
-  // the chunk is the last n_frames frames of the window, in order
-  for (int i = 0; i < n_frames; ++i)
-    if (frame_ids[n_window_frames - n_frames + i] != start_frame + i) return RKV_ERR_ARG;
   const bool abs_mode = rope_mode == RKV_ROPE_ABSOLUTE;
-  const long long base = static_cast<long long>(start_frame) + n_frames - window_frames;
-  int max_id = 0;
+  // the window is held in logical order: ids strictly increasing, the chunk's n_frames last
   for (int i = 0; i < n_window_frames; ++i) {
     if (frame_ids[i] < 0) return RKV_ERR_ARG;
-    max_id = frame_ids[i] > max_id ? frame_ids[i] : max_id;
+    if (i > 0 && frame_ids[i] <= frame_ids[i - 1]) return RKV_ERR_ARG;
   }
+  for (int i = 0; i < n_frames; ++i)
+    if (frame_ids[n_window_frames - n_frames + i] != start_frame + i) return RKV_ERR_ARG;
+  // relative mode: the caller's window cannot hold more frames than the window size
+  if (!abs_mode && n_window_frames > window_frames) return RKV_ERR_ARG;
+  const int max_id = frame_ids[n_window_frames - 1];
   if (abs_mode && max_id >= kNoAllocMaxTime) return RKV_ERR_UNSUPPORTED;
+  if (!abs_mode && window_frames > kNoAllocMaxTime) return RKV_ERR_UNSUPPORTED;  // time-table rows
+  // one rotation launch: the query run plus one run per block of consecutive frames
+  int key_runs = 1;
+  for (int i = 1; i < n_window_frames; ++i) key_runs += frame_ids[i] != frame_ids[i - 1] + 1;
+  if (1 + key_runs > kMaxRuns) return RKV_ERR_UNSUPPORTED;
+  const long long base = static_cast<long long>(start_frame) + n_frames - window_frames;
 
   const int T = tokens_per_frame, pt = 22, ph = 21, pw = 21;
   const int n_t = abs_mode ? max_id + 1 : window_frames;
   const long long Lq = static_cast<long long>(n_frames) * T;
   const long long Lk = static_cast<long long>(n_window_frames) * T;
+  // every row of every head takes 256 bytes of the array: bound the counts before the sizes
+  const long long max_rows = static_cast<long long>(kStaticScratchBytes / (kHeadDim * 2));
+  if (Lk > max_rows || static_cast<long long>(H) > max_rows || Lk * H > max_rows || grid_h > max_rows ||
+      grid_w > max_rows)
+    return RKV_ERR_CAPACITY;
   const size_t off_tab = 256;
-  const size_t tab_b = static_cast<size_t>(n_t * pt + grid_h * ph + grid_w * pw) * sizeof(float2);
+  const size_t tab_b = (static_cast<size_t>(n_t) * pt + static_cast<size_t>(grid_h) * ph +
+                        static_cast<size_t>(grid_w) * pw) * sizeof(float2);
   const size_t off_q = align256(off_tab + tab_b);
   const size_t off_k = align256(off_q + static_cast<size_t>(H) * Lq * kHeadDim * 2);
   const size_t end = align256(off_k + static_cast<size_t>(H) * Lk * kHeadDim * 2);
@@ -183,7 +197,6 @@ extern "C" __attribute__((visibility("default"))) int rkv_chunk_attention_noallo
   for (int a = 0; a < n_window_frames;) {
     int b = a + 1;
     while (b < n_window_frames && frame_ids[b] == frame_ids[b - 1] + 1) ++b;
-    if (p.n_runs == kMaxRuns) return RKV_ERR_UNSUPPORTED;
     FrameRun r;
     std::memset(&r, 0, sizeof(r));
     r.src = static_cast<const uint16_t*>(k_window);

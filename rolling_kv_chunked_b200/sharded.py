@@ -35,9 +35,11 @@ HEAD_DIM = 128
 class HeadShardedRollingKV:
     def __init__(self, layers: int, H: int, d: int, tokens_per_frame: int, window_frames: int,
                  sink_frames: int, rope_mode: int, group=None, world_size: int | None = None,
-                 rank: int | None = None, local=None):
+                 rank: int | None = None, local=None, copy_fn=None):
         """One rank of g. ``world_size`` / ``rank`` default to the process group's; ``local`` is
-        the per-rank cache of H/g heads (by default a RollingKV with this library's kernels)."""
+        the per-rank cache of H/g heads (by default a RollingKV with this library's kernels);
+        ``copy_fn(runs, n_heads, stream)`` executes the strided head-block copies that ``pack``
+        and ``unpack`` describe (by default ``rkv_copy_heads``)."""
         import torch.distributed as dist
         if d != HEAD_DIM:
             raise ValueError("head dimension must be 128")
@@ -49,6 +51,7 @@ class HeadShardedRollingKV:
         self.H, self.Hl, self.d, self.T = H, H // self.g, d, tokens_per_frame
         self.local = local if local is not None else RollingKV(layers, self.Hl, d, tokens_per_frame,
                                                                window_frames, sink_frames, rope_mode)
+        self.copy_fn = copy_fn if copy_fn is not None else copy_heads
 
     # ------------------------------------------------------------------ setup
     def set_rope_grid(self, grid_h: int, grid_w: int, theta: float = 1.0e4, pairs=(22, 21, 21)) -> None:
@@ -73,7 +76,7 @@ class HeadShardedRollingKV:
         es = x.element_size()
         runs = [(x.data_ptr() + r * self.Hl * self.d * es, send[r].data_ptr(), self.H * self.d, self.d,
                  self.Hl * self.d, self.d, Lb) for r in range(self.g)]
-        copy_heads(runs, self.Hl, stream)
+        self.copy_fn(runs, self.Hl, stream)
         return send
 
     def unpack(self, recv: torch.Tensor, out: torch.Tensor, n_frames: int, stream=None) -> None:
@@ -84,7 +87,7 @@ class HeadShardedRollingKV:
         es = out.element_size()
         runs = [(recv[r].data_ptr(), out.data_ptr() + r * self.Hl * self.d * es, self.Hl * self.d, self.d,
                  self.H * self.d, self.d, Lb) for r in range(self.g)]
-        copy_heads(runs, self.Hl, stream)
+        self.copy_fn(runs, self.Hl, stream)
 
     def attend(self, layer: int, q_heads, k_heads, v_heads, n_frames: int, start_frame: int, commit: bool,
                stream=None) -> torch.Tensor:

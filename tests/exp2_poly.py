@@ -12,7 +12,7 @@ special-function unit:
 * 2^x = 2^r * 2^f by adding r << 23 to the bit pattern of the polynomial value
   (the bits of M vanish under the shift).
 
-Run ``python rolling_kv_chunked_b200/exp2_poly.py`` to print the coefficients
+Run ``python tests/exp2_poly.py`` to print the coefficients
 and the error bound; ``EXP2_POLY3`` below are the values compiled into
 ``csrc/rkv_attention.cu`` (rounded to fp32). The maximum relative error,
 7.5e-5, is far below the 2^-9 relative rounding of the bf16 probabilities the

@@ -7,7 +7,7 @@ import os
 import numpy as np
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-_spec = importlib.util.spec_from_file_location("exp2_poly", os.path.join(ROOT, "rolling_kv_chunked_b200", "exp2_poly.py"))
+_spec = importlib.util.spec_from_file_location("exp2_poly", os.path.join(ROOT, "tests", "exp2_poly.py"))
 exp2_poly = importlib.util.module_from_spec(_spec)
 _spec.loader.exec_module(exp2_poly)
 

@@ -4,18 +4,25 @@ Each emulated rank is a HeadShardedRollingKV (its own caches of H/2 heads); the 
 with this library's kernels (rkv_copy_heads packs / unpacks the head blocks, the chunk
 attention runs per rank) and the all-to-all between the ranks is done in-process by the
 test (copies of the ranks' send slices; no collective, nothing waits on another rank).
-Checked against one unsharded RollingKV of all heads on the same inputs, at a small shape and
-at the ABot shape (24 heads, 880 tokens per frame, window 21 with 5 sinks): every output
-block bit for bit, through sinks, warm-up, eviction and wrap, both RoPE modes, and the x0 /
-renoise step on each rank's latent block bit for bit against the unsharded fused epilogue;
-the caches of each rank equal the unsharded cache's heads bit for bit; rkv_copy_heads
-against numpy slicing and its argument errors.
+At a small shape and at the ABot shape (24 heads, 880 tokens per frame, window 21 with 5
+sinks), through sinks, warm-up, eviction and wrap, in both RoPE modes:
+
+* every rank's output block is compared element by element with the fp64 oracle at the
+  attention tolerance (the small shape on all heads and rows, the ABot shape on sampled
+  heads of both ranks and sampled rows of every block), and the x0 / renoise step on each
+  rank's latent block is bit-exact against the oracle's step on the same values;
+* every output block and epilogue is also bit-identical to one unsharded RollingKV of all
+  heads on the same inputs, and each rank's cache equals the unsharded cache's heads.
+
+rkv_copy_heads against numpy slicing and its argument errors are checked as well.
 """
 import numpy as np
 import pytest
 
 import synth
-from rollout import to_bits
+from oracle import flow as oflow
+from oracle.layer import OracleLayer
+from rollout import assert_close, sample_rows, to_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -32,10 +39,24 @@ G = 2
 SHAPES = {"small": (4, 8, 10, 2, 6, 2, 5), "abot": (24, 22, 40, 3, 21, 5, 7)}
 
 
+# heads the oracle follows at each shape (both ranks' head ranges), and rows sampled per call
+ORACLE_HEADS = {"small": None, "abot": [0, 5, 11, 12, 17, 23]}
+
+
 def _dev(key, shape):
     t = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
     synth.fill_normal_bf16_cuda(t.data_ptr(), t.numel(), key, 0, torch.cuda.current_stream().cuda_stream)
     return t
+
+
+def _host(key, n_tok, H, heads):
+    """The same seeded bits on the host, [n_tok, len(heads), 128] (all heads if heads is None)."""
+    if heads is None:
+        return synth.normal_bf16_bits(key, 0, n_tok * H * 128).reshape(n_tok, H, 128)
+    t = np.arange(n_tok, dtype=np.int64)[:, None, None]
+    h = np.asarray(heads, dtype=np.int64)[None, :, None]
+    c = np.arange(128, dtype=np.int64)[None, None, :]
+    return synth.normal_bf16_bits_at(key, (t * H + h) * 128 + c)
 
 
 def _exchange(sends):
@@ -54,7 +75,7 @@ def _sharded_call(ranks, H, *tensors, n_frames):
 
 @pytest.mark.parametrize("shape", sorted(SHAPES))
 @pytest.mark.parametrize("mode", [rkv.ROPE_ABSOLUTE, rkv.ROPE_RELATIVE])
-def test_two_emulated_ranks_match_unsharded_bit_for_bit(mode, shape):
+def test_two_emulated_ranks_match_oracle_and_unsharded(mode, shape):
     H, GH, GW, C, W, S, n_chunks = SHAPES[shape]
     T = GH * GW
     ranks = [HeadShardedRollingKV(1, H, 128, T, W, S, mode, world_size=G, rank=r) for r in range(G)]
@@ -63,6 +84,9 @@ def test_two_emulated_ranks_match_unsharded_bit_for_bit(mode, shape):
         h.set_rope_grid(GH, GW)
     Lq = C * T
     Lb = Lq // G
+    oh = ORACLE_HEADS[shape]
+    orc = OracleLayer(H if oh is None else len(oh), 128, T, GH, GW, W, S, mode)
+    hsel = list(range(H)) if oh is None else oh
 
     def blocks(x, n_tok):
         b = n_tok // G
@@ -74,6 +98,7 @@ def test_two_emulated_ranks_match_unsharded_bit_for_bit(mode, shape):
     for r in range(G):
         ranks[r].local.write_chunk(0, k_in[r], v_in[r], S, 0)
     full.write_chunk(0, kr, vr, S, 0)
+    orc.write_chunk(_host(synth.stream_key(6, 1), S * T, H, oh), _host(synth.stream_key(6, 2), S * T, H, oh), S, 0)
     f0 = S
     sig = [1.0, 0.75]
     for chunk in range(n_chunks):
@@ -93,17 +118,29 @@ def test_two_emulated_ranks_match_unsharded_bit_for_bit(mode, shape):
             qs, ks, vs = _sharded_call(ranks, H, blocks(q, Lq), blocks(k, Lq), blocks(v, Lq), n_frames=C)
             outs_h = [ranks[r].attend(0, qs[r], ks[r], vs[r], C, f0, commit) for r in range(G)]
             back = _exchange([o.view(G, Lb, H // G, 128) for o in outs_h])
+            # the oracle on the same seeded inputs (sampled rows at the ABot shape)
+            rows = None if oh is None else sample_rows(Lq, n=64, seed=chunk * 2 + call)
+            ref = orc.chunk_attention(*(_host(synth.stream_key(6, 4, chunk, call, t), Lq, H, oh) for t in range(3)),
+                                      C, f0, commit, rows=rows)
+            rows_all = np.arange(Lq) if rows is None else rows
             for r in range(G):
                 out_r = torch.empty((Lb, H, 128), dtype=torch.bfloat16, device="cuda")
                 ranks[r].unpack(back[r], out_r, C)
                 torch.cuda.synchronize()
-                assert np.array_equal(to_bits(out_r), to_bits(out_full[r * Lb:(r + 1) * Lb])), (mode, chunk, call, r)
+                got_r = to_bits(out_r)
+                assert np.array_equal(got_r, to_bits(out_full[r * Lb:(r + 1) * Lb])), (mode, chunk, call, r)
+                mine = (rows_all >= r * Lb) & (rows_all < (r + 1) * Lb)
+                assert_close(got_r[rows_all[mine] - r * Lb][:, hsel], ref[mine],
+                             f"{shape} mode {mode} chunk {chunk} call {call} rank {r} vs oracle")
                 if not commit:
                     xb = xt[r * Lb:(r + 1) * Lb].contiguous()
                     eb = eps[r * Lb:(r + 1) * Lb].contiguous()
                     x0_r, xn_r = torch.empty_like(xb), torch.empty_like(xb)
                     rkv.flow_x0_renoise(xb, out_r.view(Lb, H * 128), eb, sig[0], sig[1], x0_r, xn_r)
                     torch.cuda.synchronize()
+                    rx0, rxn = oflow.x0_renoise_bf16(to_bits(xb), got_r.reshape(Lb, H * 128), to_bits(eb),
+                                                     sig[0], sig[1])
+                    assert np.array_equal(to_bits(x0_r), rx0) and np.array_equal(to_bits(xn_r), rxn)
                     assert np.array_equal(to_bits(x0_r), to_bits(x0_full[r * Lb:(r + 1) * Lb]))
                     assert np.array_equal(to_bits(xn_r), to_bits(xn_full[r * Lb:(r + 1) * Lb]))
         f0 += C

@@ -2,9 +2,12 @@
 two gloo ranks run HeadShardedRollingKV.chunk_attention / write_chunk with the real
 all-to-all (torch.distributed over gloo) around a per-rank oracle cache of H/2 heads.
 
-The CUDA copy kernel that packs and unpacks head blocks is replaced by a plain torch copy
-(a test double, CPU only), and the per-rank attention by the fp64 oracle of that rank's
-heads. Checked: every rank's output block equals the oracle of all heads on that token
+The head-block copies that pack and unpack the exchange run on the CPU: the exact run
+descriptors (pointers, strides, token counts) that HeadShardedRollingKV hands to
+rkv_copy_heads are executed by a host interpreter of that call's definition (head vector
+(t, h) of 128 bf16 moves from src + t * src_tok_stride + h * src_head_stride to the same
+offsets in dst), a test double for the CUDA copy kernel; the per-rank attention is the fp64
+oracle of that rank's heads. Checked: every rank's output block equals the oracle of all heads on that token
 block (to bf16 rounding), through sinks written with write_chunk, warm-up, eviction and
 wrap, in both RoPE modes; a head count the ranks do not divide is refused.
 """
@@ -62,17 +65,16 @@ def _worker(rank, world, port, mode, q):
             ref = self.orc.chunk_attention(to_bits(q), to_bits(k), to_bits(v), n_frames, start_frame, commit)
             out.copy_(from_bits(bf16.from_f64(ref)))
 
-    class CpuCopies(HeadShardedRollingKV):
-        """pack / unpack as plain torch copies (stand-ins for the CUDA copy kernel)."""
-        def pack(self, x, n_frames, stream=None):
-            Lb = self.block_tokens(n_frames)
-            return x.view(Lb, self.g, self.Hl, self.d).permute(1, 0, 2, 3).contiguous()
+    def host_copy_heads(runs, n_heads, stream=None):
+        """rkv_copy_heads' definition on host memory: (src, dst, src_tok_stride, src_head_stride,
+        dst_tok_stride, dst_head_stride, n_tok), strides in bf16 elements, 128-element vectors."""
+        import ctypes
+        for src, dst, sts, shs, dts, dhs, n_tok in runs:
+            for t in range(n_tok):
+                for h in range(n_heads):
+                    ctypes.memmove(dst + 2 * (t * dts + h * dhs), src + 2 * (t * sts + h * shs), 2 * 128)
 
-        def unpack(self, recv, out, n_frames, stream=None):
-            Lb = self.block_tokens(n_frames)
-            out.copy_(recv.permute(1, 0, 2, 3).reshape(Lb, self.H, self.d))
-
-    hs = CpuCopies(1, H, 128, T, W, S, mode, local=OracleLocal(H // world))
+    hs = HeadShardedRollingKV(1, H, 128, T, W, S, mode, local=OracleLocal(H // world), copy_fn=host_copy_heads)
     full = OracleLayer(H, 128, T, GH, GW, W, S, mode)
     Lq = C * T
     Lb = Lq // world
