@@ -92,17 +92,18 @@ def attention_source_sha256():
 
 
 def profiled_traffic(config_name):
-    """DRAM bytes per attention launch from the committed ncu record of this workload, if that
-    record was taken on the current kernel sources (same sha256), else None."""
+    """(DRAM bytes per attention launch, where from, the launch's algorithmic bytes) from the
+    committed ncu record of this workload, if that record was taken on the current kernel
+    sources (same sha256); (None, reason, None) otherwise."""
     config_name = {"long": "abot"}.get(config_name, config_name)  # the same launch shape
     rec = os.path.join(ROOT, "profiles", f"chunk_attention_{config_name}.traffic.json")
     if not os.path.exists(rec):
-        return None, None
+        return None, None, None
     with open(rec) as fh:
         r = json.load(fh)
     if r.get("kernel_sources_sha256") != attention_source_sha256():
-        return None, "kernel changed since the counters were taken"
-    return r["dram_bytes_per_launch"], os.path.relpath(rec, ROOT)
+        return None, "kernel changed since the counters were taken", None
+    return r["dram_bytes_per_launch"], os.path.relpath(rec, ROOT), r.get("algorithmic_bytes_per_launch")
 
 
 def peaks():
@@ -431,14 +432,14 @@ def measure_workload(args, name, headline):
     hbm = None if args.no_hbm or n_layers > 1 else measure_hbm_kernels(torch, rkv, synth, cfg, rank)
     cross = None if args.no_hbm or n_layers > 1 else measure_cross_attention(torch, rkv, synth, cfg, rank)
 
-    traffic, traffic_src = profiled_traffic(name)
+    traffic, traffic_src, traffic_alg = profiled_traffic(name)
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": config_record(cfg, world),
         "roofline": {"bound": "tensor", **attn, "traffic": traffic, "traffic_source": traffic_src,
-                     "kernel": "chunk_attention_kernel"},
+                     "traffic_algorithmic_bytes": traffic_alg, "kernel": "chunk_attention_kernel"},
         "frames_per_s_per_layer": C * n_layers * args.steps * world / (ms / 1e3),
         "rollout": rollout,
         "e2e": e2e,
@@ -1014,6 +1015,41 @@ def algorithmic_attention_bytes(cfg, keys, flow):
     return b
 
 
+def record_traffic(csv_path, config_name, command):
+    """Write profiles/chunk_attention_<workload>.traffic.json from an ncu CSV (metrics
+    dram__bytes_read.sum, dram__bytes_write.sum, gpu__time_duration.sum) of one attention launch
+    made with ``--isolate attention``, stamped with the sha256 of the kernel sources."""
+    import csv
+    vals = {}
+    with open(csv_path) as fh:
+        rows = [l for l in fh if l.startswith('"')]
+    for row in csv.DictReader(rows):
+        if "chunk_attention" in row["Kernel Name"]:
+            unit = row["Metric Unit"]
+            v = float(row["Metric Value"].replace(",", ""))
+            scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "ns": 1e-9, "us": 1e-6, "ms": 1e-3,
+                     "nsecond": 1e-9, "usecond": 1e-6,
+                     "msecond": 1e-3, "second": 1}.get(unit, 1)
+            vals.setdefault(row["Metric Name"], v * scale)
+    cfg = CONFIGS[config_name]
+    T = cfg["gh"] * cfg["gw"]
+    keys = cfg["W"] * T  # the isolated reads see the full window
+    rec = {"kernel": "chunk_attention_kernel", "workload": config_name,
+           "launch": "steady-state denoise read without the fused epilogue (bench.py --isolate attention)",
+           "kernel_sources": [os.path.relpath(f, ROOT) for f in ATTN_SRCS],
+           "kernel_sources_sha256": attention_source_sha256(),
+           "dram_bytes_read": int(vals["dram__bytes_read.sum"]), "dram_bytes_write": int(vals["dram__bytes_write.sum"]),
+           "dram_bytes_per_launch": int(vals["dram__bytes_read.sum"] + vals["dram__bytes_write.sum"]),
+           "algorithmic_bytes_per_launch": algorithmic_attention_bytes(cfg, keys, flow=False),
+           "duration_s_under_ncu": vals.get("gpu__time_duration.sum"), "command": command}
+    rec["traffic_over_algorithmic"] = rec["dram_bytes_per_launch"] / rec["algorithmic_bytes_per_launch"]
+    out = os.path.join(ROOT, "profiles", f"chunk_attention_{config_name}.traffic.json")
+    with open(out, "w") as fh:
+        json.dump(rec, fh, indent=1)
+        fh.write("\n")
+    print(out)
+
+
 def relaunch_ranks(n, impl):
     """--gpus N without a launcher: start N ranks of this same command line under
     torch.distributed.run (one process per GPU, rendezvous on 127.0.0.1) and return its exit
@@ -1050,7 +1086,13 @@ def main():
     ap.add_argument("--isolate", choices=["attention", "commit", "rope", "flow", "cross"],
                     help="only launch this kernel --reps times at the config's sizes (for profiler captures)")
     ap.add_argument("--reps", type=int, default=3, help="launches of the --isolate kernel")
+    ap.add_argument("--record-traffic", metavar="CSV",
+                    help="write the workload's attention traffic record from this ncu CSV and exit")
+    ap.add_argument("--record-command", default="", help="the ncu command the CSV came from (for the record)")
     args = ap.parse_args()
+    if args.record_traffic:
+        record_traffic(args.record_traffic, args.config, args.record_command)
+        return
     if args.isolate:
         if args.config not in CONFIGS:
             ap.error("--isolate takes one of " + ", ".join(sorted(CONFIGS)))

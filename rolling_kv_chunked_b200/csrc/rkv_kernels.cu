@@ -3,9 +3,7 @@
 //    rotation of queries, chunk keys and (relative mode) the visible window (K3);
 //  * the fp64 flow-matching x0 / renoise epilogue (K4), optionally preceded by the
 //    classifier-free guidance combine of a conditional and an unconditional prediction.
-// All move 16-byte vectors (8 bf16) per thread with grid-stride loops sized to
-// the SM count. Measured on B200 at the 720p sizes: commit copy 92 %, RoPE 84 %,
-// epilogue about 70 % of the measured HBM copy bandwidth.
+// All move 16-byte vectors (8 bf16) per thread with grid-stride loops sized to the SM count.
 #include <algorithm>
 
 #include "numeric.cuh"
@@ -99,7 +97,6 @@ __global__ void __launch_bounds__(256) frame_runs_kernel(const __grid_constant__
   }
 }
 
-// kCfg: v is the conditional prediction and u the unconditional one
 template <bool kCfg>
 __device__ __forceinline__ uint4 flow_x0(const FlowStep& step, double scale, uint4 xt, uint4 v, uint4 u, uint4 e,
                                          uint4& xn) {
@@ -108,29 +105,18 @@ __device__ __forceinline__ uint4 flow_x0(const FlowStep& step, double scale, uin
   const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
   const uint32_t ew[4] = {e.x, e.y, e.z, e.w};
   uint32_t ow[4], nw[4];
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    uint16_t o0, o1, n0 = 0, n1 = 0;
-    if (kCfg) {
-      step.apply_cfg_bits(xw[q], vw[q], uw[q], ew[q], scale, o0, n0);
-      step.apply_cfg_bits(xw[q] >> 16, vw[q] >> 16, uw[q] >> 16, ew[q] >> 16, scale, o1, n1);
-    } else {
-      step.apply_bits(xw[q], vw[q], ew[q], o0, n0);
-      step.apply_bits(xw[q] >> 16, vw[q] >> 16, ew[q] >> 16, o1, n1);
-    }
-    ow[q] = static_cast<uint32_t>(o0) | (static_cast<uint32_t>(o1) << 16);
-    nw[q] = static_cast<uint32_t>(n0) | (static_cast<uint32_t>(n1) << 16);
-  }
+  flow_vec8<kCfg>(step, scale, xw, vw, uw, ew, ow, nw);
   xn = make_uint4(nw[0], nw[1], nw[2], nw[3]);
   return make_uint4(ow[0], ow[1], ow[2], ow[3]);
 }
 
 // One 16-byte vector of each operand per thread per iteration. The bf16 <-> fp64
-// conversions run on the special-function unit and keep it busy, so HBM stays busy only
-// with many resident warps: 32 registers per thread (eight blocks of 256 threads per SM)
-// and a grid of 16 blocks per SM.
+// conversions run on the special-function unit (five per element: three in, one per
+// output, the output ones as one fp64 -> bf16 rounding each) and keep it busy, so HBM stays
+// busy only with many resident warps: 40 registers per thread (six blocks of 256 threads per
+// SM) and a grid of 16 blocks per SM.
 template <bool kCfg>
-__global__ void __launch_bounds__(256, 8) flow_kernel(const FlowParams p) {
+__global__ void __launch_bounds__(256, 6) flow_kernel(const FlowParams p) {
   FlowStep step;
   step.sigma = p.sigma;
   step.renoise = p.sigma_next >= 0.0;

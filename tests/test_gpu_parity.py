@@ -363,6 +363,56 @@ def test_score_jumps_between_key_tiles(sink_score, mode):
     h.close()
 
 
+@pytest.mark.parametrize("half", [0, 1])
+@pytest.mark.parametrize("jump", [900.0, 2000.0])
+@pytest.mark.parametrize("mode", [REL, ABS])
+def test_score_jump_inside_a_later_key_tile(half, jump, mode):
+    """One frame (128 tokens = one key tile) of the window has keys 64*half .. 64*half+63 with
+    scores `jump` above the rest, the tile not being the first of the key stream, so the
+    one-pass softmax against the running reference meets numerators far above its bound (900:
+    near 2^115, finite; 2000: beyond fp32) in one half of a later tile and must take the exact
+    path (maximum first) for that tile, with O and the row sum rescaled. The jump keys share one
+    value vector: their weights then decide nothing (the output is that vector up to the
+    other keys' vanishing weights), so the comparison is not swamped by the bf16 rounding of
+    operands this large, which moves each of their scores by several units."""
+    H, gh, gw, W, S, C = 2, 8, 16, 4, 1, 1
+    T = gh * gw
+    rng = np.random.default_rng(int(jump) + 10 * half + 100 * mode)
+    low = [p for p in range(64) if 17 <= p < 22 or 38 <= p < 43 or 59 <= p < 64]
+    dims = np.array([2 * p + e for p in low for e in (0, 1)])
+    u = np.zeros((H, 128))
+    u[:, dims] = rng.standard_normal((H, len(dims)))
+    qf = np.broadcast_to(u, (C * T, H, 128)).copy()
+
+    def bits(x):
+        return bf16.from_f64(np.asarray(x, dtype=np.float64))
+
+    def dev(b):
+        return torch.from_numpy(b.view(np.int16)).cuda().view(torch.bfloat16)
+
+    h = rkv.RollingKV(1, H, 128, T, W, S, mode)
+    h.set_rope_grid(gh, gw)
+    orc = OracleLayer(H, 128, T, gh, gw, W, S, mode)
+    qb = bits(qf)
+    for f0 in range(0, 6):
+        k = rng.standard_normal((T, H, 128))
+        v = rng.standard_normal((T, H, 128))
+        if f0 == 2:  # the frame whose half carries the jump (a later tile of the next windows)
+            k[64 * half:64 * half + 64] = jump * u / np.sum(u * u, axis=1, keepdims=True)
+            v[64 * half:64 * half + 64] = rng.standard_normal((H, 128))
+        kb, vb = bits(k), bits(v)
+        out = torch.empty((C * T, H, 128), dtype=torch.bfloat16, device="cuda")
+        for commit in (False, True):
+            h.chunk_attention(0, dev(qb), dev(kb), dev(vb), out, C, f0, commit)
+            torch.cuda.synchronize()
+            ref = orc.chunk_attention(qb, kb, vb, C, f0, commit)
+            got = to_bits(out)
+            assert np.all(np.isfinite(bf16.to_f64(got)))
+            assert_close(got, ref, f"jump {jump} half {half} frame {f0} commit {commit}")
+    assert h.poll_device_status() == rkv.OK
+    h.close()
+
+
 @pytest.mark.parametrize("mode", [REL, SLOTS, ABS])
 def test_relative_translation_invariance_bitwise(mode):
     """Identical raw window contents at two chunks whose ring layout is the same (chunks 6 and

@@ -76,12 +76,16 @@ def test_noalloc_matches_oracle_and_handle_path_twice(cfg):
         orc.write_chunk(k, v, cfg.C, f0)
         h.chunk_attention(0, _upload(q), _upload(k), _upload(v), out, cfg.C, f0, True)
         f0 += cfg.C
-    # the read: the window in logical order from the oracle's cache, then the chunk
+    # the read: the frames it attends to in logical order (the sinks and the history frames
+    # the chunk does not evict, from the oracle's cache), then the chunk itself
     qb, kb, vb = (host_bits(cfg, 0, 99, 0, t, cfg.Lq) for t in ("q", "k", "v"))
-    ids = orc.logical_frames() + list(range(f0, f0 + cfg.C))
-    assert ids == orc.window_frames(cfg.C, f0)
+    ids = orc.window_frames(cfg.C, f0)
+    held = orc.logical_frames()
+    assert ids[-cfg.C:] == list(range(f0, f0 + cfg.C)) and set(ids[:-cfg.C]) <= set(held)
     ck, cv = orc.logical_kv_bits()
-    kw, vw = _upload(np.concatenate([ck, kb])), _upload(np.concatenate([cv, vb]))
+    rows = [np.arange(held.index(f) * T, (held.index(f) + 1) * T) for f in ids[:-cfg.C]]
+    sel = np.concatenate(rows) if rows else np.zeros(0, dtype=np.int64)
+    kw, vw = _upload(np.concatenate([ck[sel], kb])), _upload(np.concatenate([cv[sel], vb]))
     ref = orc.chunk_attention(qb, kb, vb, cfg.C, f0, False)
     q = _upload(qb)
     handle_out = torch.empty((cfg.Lq, cfg.H, 128), dtype=torch.bfloat16, device="cuda")
