@@ -1020,17 +1020,29 @@ def record_traffic(csv_path, config_name, command):
     dram__bytes_read.sum, dram__bytes_write.sum, gpu__time_duration.sum) of one attention launch
     made with ``--isolate attention``, stamped with the sha256 of the kernel sources."""
     import csv
+    scales = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "ns": 1e-9, "us": 1e-6, "ms": 1e-3,
+              "nsecond": 1e-9, "usecond": 1e-6, "msecond": 1e-3, "second": 1}
     vals = {}
     with open(csv_path) as fh:
         rows = [l for l in fh if l.startswith('"')]
-    for row in csv.DictReader(rows):
-        if "chunk_attention" in row["Kernel Name"]:
-            unit = row["Metric Unit"]
-            v = float(row["Metric Value"].replace(",", ""))
-            scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "ns": 1e-9, "us": 1e-6, "ms": 1e-3,
-                     "nsecond": 1e-9, "usecond": 1e-6,
-                     "msecond": 1e-3, "second": 1}.get(unit, 1)
-            vals.setdefault(row["Metric Name"], v * scale)
+    if '"Metric Name"' in rows[0]:
+        # one metric per row (ncu --csv --log-file of a --metrics capture)
+        for row in csv.DictReader(rows):
+            if "chunk_attention" in row["Kernel Name"]:
+                v = float(row["Metric Value"].replace(",", ""))
+                vals.setdefault(row["Metric Name"], v * scales.get(row["Metric Unit"], 1))
+    else:
+        # one launch per row after a row of units (ncu -i <report> --page raw --csv)
+        table = list(csv.reader(rows))
+        hdr, units = table[0], table[1]
+        for row in table[2:]:
+            if "chunk_attention" in row[hdr.index("Kernel Name")]:
+                for h, u, v in zip(hdr, units, row):
+                    try:
+                        vals.setdefault(h, float(v.replace(",", "")) * scales.get(u, 1))
+                    except ValueError:
+                        pass
+                break
     cfg = CONFIGS[config_name]
     T = cfg["gh"] * cfg["gw"]
     keys = cfg["W"] * T  # the isolated reads see the full window
