@@ -520,3 +520,42 @@ def test_flow_epilogue_all_finite_bit_patterns():
         assert np.array_equal(to_bits(x0), rx0), s
         if sn >= 0:
             assert np.array_equal(to_bits(xn), rxn), s
+
+
+def test_chained_calls_see_their_predecessors_writes():
+    """Calls are asynchronous on the caller's stream. Chains of calls where each launch reads
+    what the previous one wrote, issued back to back without a host synchronisation, must give
+    bit for bit what the same calls give with a synchronisation after each: RoPE applied in
+    place three times (ABot chunk size), and four x0 / renoise steps each feeding the next."""
+    H, gh, gw, n_frames = 24, 22, 40, 3
+    T = gh * gw
+    h = rkv.RollingKV(1, H, 128, T, 21, 5, ABS)
+    h.set_rope_grid(gh, gw)
+    x0 = _dev_bits(synth.stream_key(11, 1), n_frames * T * H * 128).view(n_frames * T, H, 128)
+    chained, synced = x0.clone(), x0.clone()
+    for k in range(3):
+        h.rope_apply(chained, n_frames, 5 + k, 0)
+    for k in range(3):
+        h.rope_apply(synced, n_frames, 5 + k, 0)
+        torch.cuda.synchronize()
+    torch.cuda.synchronize()
+    assert np.array_equal(to_bits(chained), to_bits(synced))
+    assert not np.array_equal(to_bits(chained), to_bits(x0))
+    h.close()
+
+    n = n_frames * T * H * 128
+    v, eps = (_dev_bits(synth.stream_key(11, 2 + i), n) for i in range(2))
+    xt = _dev_bits(synth.stream_key(11, 4), n)
+    sig = [1.0, 0.75, 0.5, 0.25, -1.0]
+    outs = {}
+    for mode in ("chained", "synced"):
+        cur = xt.clone()
+        for s in range(4):
+            x0b, xn = torch.empty_like(cur), torch.empty_like(cur)
+            rkv.flow_x0_renoise(cur, v, eps, sig[s], sig[s + 1], x0b, xn if sig[s + 1] >= 0 else None)
+            if mode == "synced":
+                torch.cuda.synchronize()
+            cur = xn if sig[s + 1] >= 0 else x0b
+        torch.cuda.synchronize()
+        outs[mode] = to_bits(cur)
+    assert np.array_equal(outs["chained"], outs["synced"])
