@@ -74,9 +74,9 @@ enum : int {
   kBarVEmpty = 7,  // +stage
   kBarSFull = 9,   // +tile (0, 1)
   kBarPFull = 11,  // +tile
-  kBarODone = 13,
-  kBarDrain = 14,
-  kNumBars = 15
+  kBarODone = 13,  // short-stream form: +tile, each tile's output final on its own
+  kBarDrain = 15,
+  kNumBars = 16
 };
 
 // TMEM column of the S / P tile and of the O accumulator of query tile t (0 or 1).
@@ -223,10 +223,16 @@ __device__ __forceinline__ void scale_o(uint32_t tO, float f) {
   }
 }
 
+// kStaged (the form for short key streams, e.g. cross-attention over a few hundred text
+// tokens, where the per-CTA epilogue is a large share of the time): the output tile leaves
+// through shared memory by TMA stores, and query tile 0's epilogue starts as soon as its own
+// last value products complete. Long streams keep one-row-per-thread stores (the staged form
+// measured ~1 % slower there).
+template <bool kStaged>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                            const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_vn,
-                           const __grid_constant__ AttnParams p) {
+                           const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSmemBar);
@@ -249,6 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_init(&bars[kBarPFull + s], kBM);
     }
     ptx::mbar_init(&bars[kBarODone], 1);
+    if constexpr (kStaged) ptx::mbar_init(&bars[kBarODone + 1], 1);
     ptx::mbar_init(&bars[kBarDrain], 1);
     ptx::fence_mbar_init();
   }
@@ -269,6 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::prefetch_tmap(&tm_k);
       ptx::prefetch_tmap(&tm_vc);
       ptx::prefetch_tmap(&tm_vn);
+      if constexpr (kStaged) ptx::prefetch_tmap(&tm_o);
       ptx::mbar_arrive_expect_tx(&bars[kBarQ], 2 * kTile);
       for (int t = 0; t < 2; ++t)
         for (int c = 0; c < 2; ++c)
@@ -349,8 +357,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         k_ready = j + 1 < n_tiles && ptx::mbar_try_wait(&bars[kBarKFull + (s ^ 1)], ((j + 1) >> 1) & 1);
         if (!issue_pv(0, j)) { ok = false; break; }
       }
-      if (ok && !issue_pv(1, n_tiles - 1)) ok = false;
-      if (ok) ptx::mma_commit(&bars[kBarODone]);
+      if constexpr (kStaged) {
+        // query tile 0's output is final after PV0(last): its epilogue overlaps the last
+        // softmax and value products of tile 1
+        if (ok) ptx::mma_commit(&bars[kBarODone + 0]);
+        if (ok && !issue_pv(1, n_tiles - 1)) ok = false;
+        if (ok) ptx::mma_commit(&bars[kBarODone + 1]);
+      } else {
+        if (ok && !issue_pv(1, n_tiles - 1)) ok = false;
+        if (ok) ptx::mma_commit(&bars[kBarODone]);
+      }
       if (!ok) atomicOr(p.status, kStatusTimeout);
       // everything issued must complete before TMEM is released
       ptx::mma_commit(&bars[kBarDrain]);
@@ -495,15 +511,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_arrive(&bars[kBarPFull + wg]);
     }
     if (ok) {
-      ok = ptx::mbar_wait(&bars[kBarODone], 0, limit);
+      ok = ptx::mbar_wait(&bars[kBarODone + (kStaged ? wg : 0)], 0, limit);
       ok = __all_sync(0xffffffffu, ok);
     }
     if (!ok) {
       if (lane == 0) atomicOr(p.status, kStatusTimeout);
     } else {
       ptx::tc_fence_after();
-      const int row = m0 + wg * kBM + r;
+      const int row0 = m0 + wg * kBM;
+      const int row = row0 + r;
       const bool live = row < p.Lq;
+      // Staged form: the bf16 output tile goes to this tile's query buffer (free now: every
+      // product that reads it has completed) in the 128-byte swizzled layout of the query load
+      // (16-byte chunk k of row r at position k ^ (r mod 8)), then leaves by one TMA store per
+      // 64-column half; rows at or past Lq lie outside the output tensor and are not written.
+      uint8_t* ostage = smem + kSmemQ + wg * kTile;
       const float inv_l = 1.0f / l;
       const long long base = (static_cast<long long>(row) * p.H + head) * kHeadDim;
       FlowStep step;
@@ -515,14 +537,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < 4; ++c) {
         uint32_t rr[32];
         ptx::tmem_ld32(tO + 32 * c, rr);
-        if (live) {
-          uint32_t ob[16];
+        uint32_t ob[16];
+        if (kStaged || live) {
 #pragma unroll
           for (int i = 0; i < 16; ++i)
             ob[i] = pack_bf16x2(__uint_as_float(rr[2 * i]) * inv_l, __uint_as_float(rr[2 * i + 1]) * inv_l);
-          uint4* dst = reinterpret_cast<uint4*>(p.out + base + 32 * c);
+        }
+        if constexpr (kStaged) {
+          uint8_t* orow = ostage + (c >> 1) * kSlab + r * 128;
 #pragma unroll
-          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(ob[4 * v], ob[4 * v + 1], ob[4 * v + 2], ob[4 * v + 3]);
+          for (int v = 0; v < 4; ++v)
+            *reinterpret_cast<uint4*>(orow + (((((c & 1) << 2) + v) ^ (r & 7)) << 4)) =
+                make_uint4(ob[4 * v], ob[4 * v + 1], ob[4 * v + 2], ob[4 * v + 3]);
+        }
+        if (live) {
+          if constexpr (!kStaged) {
+            uint4* dst = reinterpret_cast<uint4*>(p.out + base + 32 * c);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(ob[4 * v], ob[4 * v + 1], ob[4 * v + 2], ob[4 * v + 3]);
+          }
           if (p.flow) {
             const uint4* xtp = reinterpret_cast<const uint4*>(p.xt + base + 32 * c);
             const uint4* ep = reinterpret_cast<const uint4*>(p.eps + base + 32 * c);
@@ -561,6 +594,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      if constexpr (kStaged) {
+        ptx::fence_proxy_async_smem();
+        ptx::named_bar_sync(1 + wg, kBM);
+        if (r == 0 && row0 < p.Lq) {
+          ptx::tma_store_3d(&tm_o, ostage, 0, head, row0);
+          ptx::tma_store_3d(&tm_o, ostage + kSlab, 64, head, row0);
+          ptx::bulk_commit_group();
+          ptx::bulk_wait_read_all();  // the buffer must stay until the copy has read it
+        }
+      }
     }
   }
 
@@ -572,8 +615,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
+// Key streams of at most this many 128-key tiles take the staged-epilogue form.
+constexpr int kShortStreamTiles = 16;
+
 cudaError_t launch_attention(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_vc,
-                             const CUtensorMap& tm_vn, const AttnParams& p, cudaStream_t stream) {
+                             const CUtensorMap& tm_vn, const CUtensorMap& tm_o, const AttnParams& p,
+                             cudaStream_t stream) {
   // the dynamic shared-memory limit is a per-device setting: raised once on every device
   // this process launches on, whichever host thread gets there first
   constexpr int kMaxDevices = 64;
@@ -586,13 +633,20 @@ cudaError_t launch_attention(const CUtensorMap& tm_q, const CUtensorMap& tm_k, c
   {
     std::lock_guard<std::mutex> lock(mu);
     if (!configured[dev]) {
-      err = cudaFuncSetAttribute(chunk_attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+      err = cudaFuncSetAttribute(chunk_attention_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kSmemBytes);
+      if (err == cudaSuccess)
+        err = cudaFuncSetAttribute(chunk_attention_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   kSmemBytes);
       if (err != cudaSuccess) return err;
       configured[dev] = true;
     }
   }
   dim3 grid((p.Lq + 2 * kBM - 1) / (2 * kBM), p.H);
-  chunk_attention_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_q, tm_k, tm_vc, tm_vn, p);
+  if (p.n_tiles <= kShortStreamTiles)
+    chunk_attention_kernel<true><<<grid, kThreads, kSmemBytes, stream>>>(tm_q, tm_k, tm_vc, tm_vn, tm_o, p);
+  else
+    chunk_attention_kernel<false><<<grid, kThreads, kSmemBytes, stream>>>(tm_q, tm_k, tm_vc, tm_vn, tm_o, p);
   return cudaGetLastError();
 }
 

@@ -536,11 +536,13 @@ int chunk_attention_impl(rkv_handle h, int layer, const void* q, const void* k, 
   }
   ap.status = h->status;
   ap.wait_limit_ns = h->wait_ns;
-  CUtensorMap tm_vn;
-  if (!encode_token_major(&tm_vn, v, C * T, h->H, rkv::kKeyBox)) return RKV_ERR_CUDA;
+  CUtensorMap tm_vn, tm_o;
+  if (!encode_token_major(&tm_vn, v, C * T, h->H, rkv::kKeyBox) ||
+      !encode_token_major(&tm_o, out, C * T, h->H, rkv::kQueryBox))
+    return RKV_ERR_CUDA;
   const bool timed = h->timing && h->timing_n < h->timing_max;
   if (timed && cudaEventRecord(h->ev_start[h->timing_n], st) != cudaSuccess) return RKV_ERR_CUDA;
-  rc = cuda_rc(rkv::launch_attention(L.tm_q, L.tm_k, L.tm_vc, tm_vn, ap, st));
+  rc = cuda_rc(rkv::launch_attention(L.tm_q, L.tm_k, L.tm_vc, tm_vn, tm_o, ap, st));
   if (rc) return rc;
   if (timed) {
     if (cudaEventRecord(h->ev_stop[h->timing_n], st) != cudaSuccess) return RKV_ERR_CUDA;
@@ -655,11 +657,13 @@ RKV_API int rkv_cross_attention(rkv_handle h, int layer, const void* q, void* ou
   ap.sigma_next = -1.0;
   ap.status = h->status;
   ap.wait_limit_ns = h->wait_ns;
-  CUtensorMap tm_q;
-  if (!encode_token_major(&tm_q, q, n_tokens, h->H, rkv::kQueryBox)) return RKV_ERR_CUDA;
+  CUtensorMap tm_q, tm_o;
+  if (!encode_token_major(&tm_q, q, n_tokens, h->H, rkv::kQueryBox) ||
+      !encode_token_major(&tm_o, out, n_tokens, h->H, rkv::kQueryBox))
+    return RKV_ERR_CUDA;
   const bool timed = h->timing && h->timing_n < h->timing_max;
   if (timed && cudaEventRecord(h->ev_start[h->timing_n], st) != cudaSuccess) return RKV_ERR_CUDA;
-  rc = cuda_rc(rkv::launch_attention(tm_q, L.tm_tk, L.tm_tv, L.tm_tv, ap, st));
+  rc = cuda_rc(rkv::launch_attention(tm_q, L.tm_tk, L.tm_tv, L.tm_tv, tm_o, ap, st));
   if (rc) return rc;
   if (timed) {
     if (cudaEventRecord(h->ev_stop[h->timing_n], st) != cudaSuccess) return RKV_ERR_CUDA;

@@ -68,7 +68,8 @@ cudaError_t launch_flow(const FlowParams& p, cudaStream_t stream);
 // ---------------------------------------------------------------- attention
 // One key segment: K rows [k_row0, k_row0 + n_rows) of the rotated-K buffer and
 // V rows [v_row0, ...) of either the cache V ring (src 0) or the caller's v (src 1).
-// tm_q must use boxes of kQueryBox rows; tm_k, tm_vc and tm_vn boxes of kKeyBox rows.
+// tm_q and tm_o must use boxes of kQueryBox rows; tm_k, tm_vc and tm_vn boxes of kKeyBox rows.
+// tm_o maps the output [Lq][H][d] token-major (coordinates x, head, row).
 struct AttnSeg {
   int src;
   int k_row0;
@@ -100,6 +101,7 @@ struct AttnParams {
 };
 
 cudaError_t launch_attention(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_vc,
-                             const CUtensorMap& tm_vn, const AttnParams& p, cudaStream_t stream);
+                             const CUtensorMap& tm_vn, const CUtensorMap& tm_o, const AttnParams& p,
+                             cudaStream_t stream);
 
 }  // namespace rkv

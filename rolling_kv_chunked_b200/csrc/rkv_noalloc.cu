@@ -215,8 +215,9 @@ extern "C" __attribute__((visibility("default"))) int rkv_chunk_attention_noallo
   rc = launch_frame_runs(p, static_cast<int>(Lk > Lq ? Lk : Lq), st) == cudaSuccess ? RKV_OK : RKV_ERR_CUDA;
   if (rc != RKV_OK) return rc;
 
-  CUtensorMap tm_q, tm_k, tm_v;
+  CUtensorMap tm_q, tm_k, tm_v, tm_o;
   if (!encode(&tm_q, qs, Lq, H, kHeadDim * 2, Lq * kHeadDim * 2, kQueryBox, 1) ||
+      !encode(&tm_o, out, H, Lq, kHeadDim * 2, static_cast<uint64_t>(H) * kHeadDim * 2, 1, kQueryBox) ||
       !encode(&tm_k, ks, Lk, H, kHeadDim * 2, Lk * kHeadDim * 2, kKeyBox, 1) ||
       !encode(&tm_v, v_window, H, Lk, kHeadDim * 2, static_cast<uint64_t>(H) * kHeadDim * 2, 1, kKeyBox))
     return RKV_ERR_CUDA;
@@ -235,5 +236,5 @@ extern "C" __attribute__((visibility("default"))) int rkv_chunk_attention_noallo
   ap.sigma_next = -1.0;
   ap.status = status;
   ap.wait_limit_ns = 2000000000ull;
-  return launch_attention(tm_q, tm_k, tm_v, tm_v, ap, st) == cudaSuccess ? RKV_OK : RKV_ERR_CUDA;
+  return launch_attention(tm_q, tm_k, tm_v, tm_v, tm_o, ap, st) == cudaSuccess ? RKV_OK : RKV_ERR_CUDA;
 }

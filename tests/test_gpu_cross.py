@@ -1,8 +1,9 @@
 """GPU parity of the cross-attention over the cached text K/V (through the C ABI).
 
-* ragged and tile-aligned text lengths (1, 77, 128, 512, 600) and query counts (1 .. 2 CTAs
-  with ragged tails): every element within the attention tolerance of the fp64 oracle, plus a
-  peaked-softmax case (queries x 4);
+* ragged and tile-aligned text lengths (1, 77, 128, 512, 600) and query counts (1 .. 3 CTAs
+  with ragged tails, the second 128-row tile of a CTA absent, partial or full): every element
+  within the attention tolerance of the fp64 oracle, plus a peaked-softmax case (queries x 4);
+  guard rows after the output stay untouched;
 * the ABot shape (H = 24, 2640 queries, 512 text tokens): all elements; the 720p shape
   (H = 40, 14400 queries): sampled rows of all heads;
 * interleaved with a self-attention rollout: cross calls leave the rolling cache bit-exact,
@@ -48,12 +49,16 @@ def test_cross_small_every_element(n_text):
     h.set_text_kv(0, kt, vt)
     orc = _oracle(H)
     orc.set_text_kv(ktb, vtb)
-    for n_q, scale in [(1, 1.0), (33, 1.0), (256, 1.0), (300, 1.0), (513, 1.0), (300, 4.0)]:
+    for n_q, scale in [(1, 1.0), (33, 1.0), (200, 1.0), (256, 1.0), (300, 1.0), (400, 1.0), (513, 1.0),
+                       (300, 4.0)]:
         q, qb = _pair(H, n_q, synth.stream_key(0, 71, n_text, n_q), scale)
-        out = torch.empty_like(q)
+        # the output is a view followed by 80 guard rows that no store may reach
+        full = torch.full((n_q + 80, H, 128), -7.0, dtype=torch.bfloat16, device="cuda")
+        out = full[:n_q]
         h.cross_attention(0, q, out)
         torch.cuda.synchronize()
         assert_close(to_bits(out), orc.cross_attention(qb), f"cross n_text {n_text} n_q {n_q} x{scale}")
+        assert bool((full[n_q:] == -7.0).all()), f"rows past the output written (n_text {n_text}, n_q {n_q})"
     assert h.poll_device_status() == rkv.OK
     h.close()
 

@@ -559,3 +559,46 @@ def test_chained_calls_see_their_predecessors_writes():
         torch.cuda.synchronize()
         outs[mode] = to_bits(cur)
     assert np.array_equal(outs["chained"], outs["synced"])
+
+
+@pytest.mark.parametrize("gh, gw, C, W", [(8, 10, 3, 7), (10, 20, 2, 12)])
+def test_outputs_stay_in_bounds_and_feed_the_next_call(gh, gw, C, W):
+    """Each call's output is the next call's queries, issued without a host synchronisation,
+    and the output is a view followed by guard rows. The chunk (240 / 400 queries) ends inside
+    the second 128-row tile of its last query block; the windows cover short key streams (a
+    few tiles, output written through shared memory by TMA stores) and, in the second shape,
+    long ones (up to 19 tiles, one row per thread). Outputs equal bit for bit those of the same
+    chain with a synchronisation after each call, and no guard row changes."""
+    H, S = 2, 2
+    T = gh * gw
+    Lq = C * T
+    outs = {}
+    for mode in ("chained", "synced"):
+        h = rkv.RollingKV(1, H, 128, T, W, S, ABS)
+        h.set_rope_grid(gh, gw)
+        full = torch.full((Lq + 80, H, 128), -7.0, dtype=torch.bfloat16, device="cuda")
+        q = _dev_bits(synth.stream_key(12, 1), Lq * H * 128).view(Lq, H, 128)
+        seq = []
+        for c in range(6):
+            k = _dev_bits(synth.stream_key(12, 2, c), Lq * H * 128).view(Lq, H, 128)
+            v = _dev_bits(synth.stream_key(12, 3, c), Lq * H * 128).view(Lq, H, 128)
+            out = full[:Lq]
+            h.chunk_attention(0, q, k, v, out, C, c * C, True)
+            if mode == "synced":
+                torch.cuda.synchronize()
+            q = out.clone() if mode == "synced" else _copy_on_stream(out)
+            seq.append(q)
+        torch.cuda.synchronize()
+        assert bool((full[Lq:] == -7.0).all()), f"{mode}: rows past the output written"
+        assert h.poll_device_status() == rkv.OK
+        outs[mode] = [to_bits(t) for t in seq]
+        h.close()
+    for a, b in zip(outs["chained"], outs["synced"]):
+        assert np.array_equal(a, b)
+
+
+def _copy_on_stream(t):
+    """A device copy queued on the current stream (no host synchronisation)."""
+    c = torch.empty_like(t)
+    c.copy_(t, non_blocking=True)
+    return c
