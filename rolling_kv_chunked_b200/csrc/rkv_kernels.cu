@@ -56,10 +56,14 @@ __device__ __forceinline__ uint4 rotate_vec(uint4 val, const float2 (&cs)[4]) {
 }
 
 // One warp per token. Lane l always handles the 16-byte vector l % 16 of heads
-// l / 16, l / 16 + 2, ... (eight heads in flight, their loads issued before the (cos, sin)
+// l / 16, l / 16 + 2, ... (kPer heads in flight, their loads issued before the (cos, sin)
 // lookups), so a half-warp moves one head's 256 contiguous bytes per instruction and each
-// lane fetches its four (cos, sin) pairs once per eight heads. blockIdx.y selects the run.
-__global__ void __launch_bounds__(256) frame_runs_kernel(const __grid_constant__ FrameRunParams p) {
+// lane fetches its four (cos, sin) pairs once per kPer heads. blockIdx.y selects the run.
+// kPer = 8 (blocks of 256 threads) in general; kPer = 12 (blocks of 128) when a token has
+// 17-24 heads, so that all of a token's heads are in flight at once and a launch of one
+// chunk (a few thousand tokens, every warp resident) waits on one DRAM round trip, not two.
+template <int kPer>
+__global__ void __launch_bounds__(kPer == 8 ? 256 : 128) frame_runs_kernel(const __grid_constant__ FrameRunParams p) {
   const int r = blockIdx.y;
   if (r >= p.n_runs) return;
   const FrameRun& run = p.run[r];
@@ -70,10 +74,10 @@ __global__ void __launch_bounds__(256) frame_runs_kernel(const __grid_constant__
   for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < run.n_tok; t += warps) {
     const uint16_t* src = run.src + static_cast<long long>(run.src_tok0 + t) * run.src_tok_stride + vec * 8;
     uint16_t* dst = run.dst + static_cast<long long>(run.dst_tok0 + t) * run.dst_tok_stride + vec * 8;
-    for (int hb = h0; hb < p.H; hb += 2 * 8) {
-      uint4 val[8];
+    for (int hb = h0; hb < p.H; hb += 2 * kPer) {
+      uint4 val[kPer];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < kPer; ++u) {
         const int h = hb + 2 * u;
         if (h < p.H) val[u] = __ldg(reinterpret_cast<const uint4*>(src + h * run.src_head_stride));
       }
@@ -85,7 +89,7 @@ __global__ void __launch_bounds__(256) frame_runs_kernel(const __grid_constant__
         pair_cos_sin(vec, min(max(run.t0 + frame, p.t_lo), p.t_hi), hh, tok - hh * p.grid_w, p, cs);
       }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < kPer; ++u) {
         const int h = hb + 2 * u;
         if (h < p.H) {
           uint4 v = val[u];
@@ -160,11 +164,20 @@ __global__ void __launch_bounds__(256, 6) flow_kernel(const FlowParams p) {
 
 cudaError_t launch_frame_runs(const FrameRunParams& p, int max_tok, cudaStream_t stream) {
   if (p.n_runs <= 0) return cudaSuccess;
+  const long long per_run = p.n_runs > 1 ? p.n_runs : 1;
+  if (p.H > 16 && p.H <= 24) {
+    long long blocks = (static_cast<long long>(max_tok) + 3) / 4;  // 4 warps (tokens) per block
+    const long long cap = static_cast<long long>(sm_count()) * 16 / per_run + 1;
+    blocks = std::max(1LL, std::min(blocks, cap));
+    dim3 grid(static_cast<unsigned>(blocks), static_cast<unsigned>(p.n_runs));
+    frame_runs_kernel<12><<<grid, 128, 0, stream>>>(p);
+    return cudaGetLastError();
+  }
   long long blocks = (static_cast<long long>(max_tok) + 7) / 8;  // 8 warps (tokens) per block
-  const long long cap = static_cast<long long>(sm_count()) * 8 / (p.n_runs > 1 ? p.n_runs : 1) + 1;
+  const long long cap = static_cast<long long>(sm_count()) * 8 / per_run + 1;
   blocks = std::max(1LL, std::min(blocks, cap));
   dim3 grid(static_cast<unsigned>(blocks), static_cast<unsigned>(p.n_runs));
-  frame_runs_kernel<<<grid, 256, 0, stream>>>(p);
+  frame_runs_kernel<8><<<grid, 256, 0, stream>>>(p);
   return cudaGetLastError();
 }
 
