@@ -41,6 +41,7 @@
 // Every mbarrier wait is bounded in wall time; on expiry the kernel records
 // kStatusTimeout in the status word, stops issuing work, waits (bounded) for the
 // copies and MMAs it already issued, frees TMEM and returns.
+#include <algorithm>
 #include <cfloat>
 #include <mutex>
 
@@ -74,9 +75,9 @@ enum : int {
   kBarVEmpty = 7,  // +stage
   kBarSFull = 9,   // +tile (0, 1)
   kBarPFull = 11,  // +tile
-  kBarODone = 13,  // short-stream form: +tile, each tile's output final on its own
-  kBarDrain = 15,
-  kNumBars = 16
+  kBarODone = 13,
+  kBarDrain = 14,
+  kNumBars = 15
 };
 
 // TMEM column of the S / P tile and of the O accumulator of query tile t (0 or 1).
@@ -223,16 +224,10 @@ __device__ __forceinline__ void scale_o(uint32_t tO, float f) {
   }
 }
 
-// kStaged (the form for short key streams, e.g. cross-attention over a few hundred text
-// tokens, where the per-CTA epilogue is a large share of the time): the output tile leaves
-// through shared memory by TMA stores, and query tile 0's epilogue starts as soon as its own
-// last value products complete. Long streams keep one-row-per-thread stores (the staged form
-// measured ~1 % slower there).
-template <bool kStaged>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                            const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_vn,
-                           const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ AttnParams p) {
+                           const __grid_constant__ AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSmemBar);
@@ -255,7 +250,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_init(&bars[kBarPFull + s], kBM);
     }
     ptx::mbar_init(&bars[kBarODone], 1);
-    if constexpr (kStaged) ptx::mbar_init(&bars[kBarODone + 1], 1);
     ptx::mbar_init(&bars[kBarDrain], 1);
     ptx::fence_mbar_init();
   }
@@ -276,7 +270,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::prefetch_tmap(&tm_k);
       ptx::prefetch_tmap(&tm_vc);
       ptx::prefetch_tmap(&tm_vn);
-      if constexpr (kStaged) ptx::prefetch_tmap(&tm_o);
       ptx::mbar_arrive_expect_tx(&bars[kBarQ], 2 * kTile);
       for (int t = 0; t < 2; ++t)
         for (int c = 0; c < 2; ++c)
@@ -357,16 +350,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         k_ready = j + 1 < n_tiles && ptx::mbar_try_wait(&bars[kBarKFull + (s ^ 1)], ((j + 1) >> 1) & 1);
         if (!issue_pv(0, j)) { ok = false; break; }
       }
-      if constexpr (kStaged) {
-        // query tile 0's output is final after PV0(last): its epilogue overlaps the last
-        // softmax and value products of tile 1
-        if (ok) ptx::mma_commit(&bars[kBarODone + 0]);
-        if (ok && !issue_pv(1, n_tiles - 1)) ok = false;
-        if (ok) ptx::mma_commit(&bars[kBarODone + 1]);
-      } else {
-        if (ok && !issue_pv(1, n_tiles - 1)) ok = false;
-        if (ok) ptx::mma_commit(&bars[kBarODone]);
-      }
+      if (ok && !issue_pv(1, n_tiles - 1)) ok = false;
+      if (ok) ptx::mma_commit(&bars[kBarODone]);
       if (!ok) atomicOr(p.status, kStatusTimeout);
       // everything issued must complete before TMEM is released
       ptx::mma_commit(&bars[kBarDrain]);
@@ -511,21 +496,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_arrive(&bars[kBarPFull + wg]);
     }
     if (ok) {
-      ok = ptx::mbar_wait(&bars[kBarODone + (kStaged ? wg : 0)], 0, limit);
+      ok = ptx::mbar_wait(&bars[kBarODone], 0, limit);
       ok = __all_sync(0xffffffffu, ok);
     }
     if (!ok) {
       if (lane == 0) atomicOr(p.status, kStatusTimeout);
     } else {
       ptx::tc_fence_after();
-      const int row0 = m0 + wg * kBM;
-      const int row = row0 + r;
+      const int row = m0 + wg * kBM + r;
       const bool live = row < p.Lq;
-      // Staged form: the bf16 output tile goes to this tile's query buffer (free now: every
-      // product that reads it has completed) in the 128-byte swizzled layout of the query load
-      // (16-byte chunk k of row r at position k ^ (r mod 8)), then leaves by one TMA store per
-      // 64-column half; rows at or past Lq lie outside the output tensor and are not written.
-      uint8_t* ostage = smem + kSmemQ + wg * kTile;
       const float inv_l = 1.0f / l;
       const long long base = (static_cast<long long>(row) * p.H + head) * kHeadDim;
       FlowStep step;
@@ -537,25 +516,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < 4; ++c) {
         uint32_t rr[32];
         ptx::tmem_ld32(tO + 32 * c, rr);
-        uint32_t ob[16];
-        if (kStaged || live) {
+        if (live) {
+          uint32_t ob[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i)
             ob[i] = pack_bf16x2(__uint_as_float(rr[2 * i]) * inv_l, __uint_as_float(rr[2 * i + 1]) * inv_l);
-        }
-        if constexpr (kStaged) {
-          uint8_t* orow = ostage + (c >> 1) * kSlab + r * 128;
+          uint4* dst = reinterpret_cast<uint4*>(p.out + base + 32 * c);
 #pragma unroll
-          for (int v = 0; v < 4; ++v)
-            *reinterpret_cast<uint4*>(orow + (((((c & 1) << 2) + v) ^ (r & 7)) << 4)) =
-                make_uint4(ob[4 * v], ob[4 * v + 1], ob[4 * v + 2], ob[4 * v + 3]);
-        }
-        if (live) {
-          if constexpr (!kStaged) {
-            uint4* dst = reinterpret_cast<uint4*>(p.out + base + 32 * c);
-#pragma unroll
-            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(ob[4 * v], ob[4 * v + 1], ob[4 * v + 2], ob[4 * v + 3]);
-          }
+          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(ob[4 * v], ob[4 * v + 1], ob[4 * v + 2], ob[4 * v + 3]);
           if (p.flow) {
             const uint4* xtp = reinterpret_cast<const uint4*>(p.xt + base + 32 * c);
             const uint4* ep = reinterpret_cast<const uint4*>(p.eps + base + 32 * c);
@@ -594,17 +562,431 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if constexpr (kStaged) {
-        ptx::fence_proxy_async_smem();
-        ptx::named_bar_sync(1 + wg, kBM);
-        if (r == 0 && row0 < p.Lq) {
-          ptx::tma_store_3d(&tm_o, ostage, 0, head, row0);
-          ptx::tma_store_3d(&tm_o, ostage + kSlab, 64, head, row0);
-          ptx::bulk_commit_group();
-          ptx::bulk_wait_read_all();  // the buffer must stay until the copy has read it
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  if (warp == 9) ptx::tmem_dealloc(tmem, 512);
+}
+
+
+// ---------------------------------------------------------------------------------------------
+// Short key streams (at most kShortStreamTiles tiles: the cross-attention over a prompt's text
+// tokens, the first chunks of a rollout). Each CTA stays resident and walks the units (head,
+// 256-row query block) b, b + G, b + 2G, ... (G = gridDim.x <= SM count) with one running
+// count of key tiles across units, so the stage and phase bookkeeping continues from one unit
+// to the next. What this form adds over the long-stream kernel:
+//   * the next unit's queries are loaded as soon as the current unit's last score products
+//     have completed (a Q-empty barrier committed after them), and its first score product
+//     S0 is issued before the current unit's last value product PV1, so the tensor core and
+//     the softmax pipeline run across unit boundaries instead of draining per CTA;
+//   * each query tile's epilogue starts when its own last value products complete (one
+//     output barrier per tile) and overlaps the other tile's last softmax;
+//   * the bf16 output leaves by TMA stores from a 16 KB staging buffer per query tile (one
+//     64-column half at a time, the second half's TMEM reads overlapping the first half's
+//     store), instead of one row per thread (each warp store instruction would touch 32
+//     token rows H * 256 bytes apart).
+// Warp roles, TMEM layout, the softmax and the bounded waits are those of the long-stream
+// kernel above.
+constexpr int kSmemStage = 6 * kTile;               // two 16 KB output halves, one per query tile
+constexpr int kSmemBarShort = 6 * kTile + 2 * kSlab;
+constexpr int kSmemBytesShort = kSmemBarShort + 256 + 1024;
+static_assert(kSmemBytesShort <= 232448, "short-stream form exceeds the shared-memory limit");
+
+enum : int {
+  kSbQ = 0,        // queries of the current unit landed
+  kSbQEmpty = 1,   // every score product of a unit completed: its query buffer is free
+  kSbKFull = 2,    // +stage
+  kSbKEmpty = 4,   // +stage
+  kSbVFull = 6,    // +stage
+  kSbVEmpty = 8,   // +stage
+  kSbSFull = 10,   // +tile
+  kSbPFull = 12,   // +tile
+  kSbODone = 14,   // +tile: that tile's output of the unit is final
+  kSbDrain = 16,
+  kSbCount = 17
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    chunk_attention_short_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                                 const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_vn,
+                                 const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ AttnParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSmemBarShort);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kSbCount + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const unsigned long long limit = p.wait_limit_ns;
+  const int n_qb = (p.Lq + 2 * kBM - 1) / (2 * kBM);
+  const int n_units = n_qb * p.H;
+  const int G = gridDim.x;
+  const int n_my = (n_units - static_cast<int>(blockIdx.x) + G - 1) / G;  // units of this CTA (>= 1)
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&bars[kSbQ], 1);
+    ptx::mbar_init(&bars[kSbQEmpty], 1);
+    for (int s = 0; s < 2; ++s) {
+      ptx::mbar_init(&bars[kSbKFull + s], 1);
+      ptx::mbar_init(&bars[kSbKEmpty + s], 1);
+      ptx::mbar_init(&bars[kSbVFull + s], 1);
+      ptx::mbar_init(&bars[kSbVEmpty + s], 1);
+      ptx::mbar_init(&bars[kSbSFull + s], 1);
+      ptx::mbar_init(&bars[kSbPFull + s], kBM);
+      ptx::mbar_init(&bars[kSbODone + s], 1);
+    }
+    ptx::mbar_init(&bars[kSbDrain], 1);
+    ptx::fence_mbar_init();
+  }
+  if (warp == 9) {
+    ptx::tmem_alloc(tmem_slot, 512);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int n_tiles = p.n_tiles;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      ptx::prefetch_tmap(&tm_q);
+      ptx::prefetch_tmap(&tm_k);
+      ptx::prefetch_tmap(&tm_vc);
+      ptx::prefetch_tmap(&tm_vn);
+      ptx::prefetch_tmap(&tm_o);
+      bool ok = true;
+      int nq = 0, nk = 0, nv = 0;  // loads issued (units for Q, global tiles for K and V)
+      for (int i = 0; ok && i < n_my; ++i) {
+        const int u = static_cast<int>(blockIdx.x) + i * G;
+        const int head = u / n_qb;
+        const int m0 = (u - head * n_qb) * (2 * kBM);
+        if (i > 0 && !ptx::mbar_wait(&bars[kSbQEmpty], (i - 1) & 1, limit)) { ok = false; break; }
+        ptx::mbar_arrive_expect_tx(&bars[kSbQ], 2 * kTile);
+        for (int t = 0; t < 2; ++t)
+          for (int c = 0; c < 2; ++c)
+            if (p.q_token_major)
+              ptx::tma_load_3d(smem + kSmemQ + t * kTile + c * kSlab, &tm_q, &bars[kSbQ], c * 64, head, m0 + t * kBM);
+            else
+              ptx::tma_load_3d(smem + kSmemQ + t * kTile + c * kSlab, &tm_q, &bars[kSbQ], c * 64, m0 + t * kBM, head);
+        nq = i + 1;
+        for (int j = 0; j < n_tiles; ++j) {
+          const int g = i * n_tiles + j;
+          const int s = g & 1;
+          int src, krow, vrow, valid;
+          tile_of(p, j, src, krow, vrow, valid);
+          if (g >= 2 && !ptx::mbar_wait(&bars[kSbKEmpty + s], ((g - 2) >> 1) & 1, limit)) { ok = false; break; }
+          ptx::mbar_arrive_expect_tx(&bars[kSbKFull + s], kTile);
+          for (int c = 0; c < 2; ++c)
+            ptx::tma_load_3d(smem + kSmemK + s * kTile + c * kSlab, &tm_k, &bars[kSbKFull + s], c * 64, krow, head);
+          nk = g + 1;
+          if (g >= 2 && !ptx::mbar_wait(&bars[kSbVEmpty + s], ((g - 2) >> 1) & 1, limit)) { ok = false; break; }
+          ptx::mbar_arrive_expect_tx(&bars[kSbVFull + s], kTile);
+          for (int c = 0; c < 2; ++c) {
+            if (src == 0)
+              ptx::tma_load_3d(smem + kSmemV + s * kTile + c * kSlab, &tm_vc, &bars[kSbVFull + s], c * 64, vrow, head);
+            else
+              ptx::tma_load_3d(smem + kSmemV + s * kTile + c * kSlab, &tm_vn, &bars[kSbVFull + s], c * 64, head, vrow);
+          }
+          nv = g + 1;
+        }
+      }
+      if (!ok) atomicOr(p.status, kStatusTimeout);
+      // every copy issued must land before the CTA may exit
+      if (nq > 0) ptx::mbar_wait(&bars[kSbQ], (nq - 1) & 1, kDrainNs);
+      for (int g = (nk > 2 ? nk - 2 : 0); g < nk; ++g) ptx::mbar_wait(&bars[kSbKFull + (g & 1)], (g >> 1) & 1, kDrainNs);
+      for (int g = (nv > 2 ? nv - 2 : 0); g < nv; ++g) ptx::mbar_wait(&bars[kSbVFull + (g & 1)], (g >> 1) & 1, kDrainNs);
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t q_addr[2] = {ptx::smem_u32(smem + kSmemQ), ptx::smem_u32(smem + kSmemQ + kTile)};
+      const uint32_t k_addr = ptx::smem_u32(smem + kSmemK);
+      const uint32_t v_addr = ptx::smem_u32(smem + kSmemV);
+      auto issue_s = [&](int t, uint32_t kt) {
+#pragma unroll
+        for (int kk = 0; kk < kHeadDim / 16; ++kk)
+          ptx::mma_ss(tmem + col_s(t), desc_kmajor(q_addr[t], kk), desc_kmajor(kt, kk), kIdescS, kk > 0 ? 1u : 0u);
+      };
+      // O_t += P_t(g) V(g) for global tile g, the unit's local tile index jl (0: overwrite O);
+      // V(g) already observed. Returns false if a wait expired.
+      auto issue_pv = [&](int t, int g, int jl) -> bool {
+        if (!ptx::mbar_wait(&bars[kSbPFull + t], g & 1, limit)) return false;
+        ptx::tc_fence_after();
+        const uint32_t vt = v_addr + (g & 1) * kTile;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          ptx::mma_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8, desc_v(vt, kk), kIdescPV,
+                      (jl > 0 || kk > 0) ? 1u : 0u);
+        if (t == 1) ptx::mma_commit(&bars[kSbVEmpty + (g & 1)]);
+        return true;
+      };
+      bool ok = true;
+      int g = 0;
+      bool k_ready = false;
+      for (int i = 0; ok && i < n_my; ++i) {
+        if (!ptx::mbar_wait(&bars[kSbQ], i & 1, limit)) { ok = false; break; }
+        for (int j = 0; j < n_tiles; ++j, ++g) {
+          const int s = g & 1;
+          if (!k_ready && !ptx::mbar_wait(&bars[kSbKFull + s], (g >> 1) & 1, limit)) { ok = false; break; }
+          ptx::tc_fence_after();
+          const uint32_t kt = k_addr + s * kTile;
+          issue_s(0, kt);
+          ptx::mma_commit(&bars[kSbSFull + 0]);
+          if (g > 0) {
+            // the previous tile's PV1; at j == 0 it is the previous unit's last
+            if (!issue_pv(1, g - 1, j > 0 ? j - 1 : n_tiles - 1)) { ok = false; break; }
+            if (j == 0) ptx::mma_commit(&bars[kSbODone + 1]);
+          }
+          issue_s(1, kt);
+          ptx::mma_commit(&bars[kSbSFull + 1]);
+          ptx::mma_commit(&bars[kSbKEmpty + s]);
+          if (j == n_tiles - 1) ptx::mma_commit(&bars[kSbQEmpty]);
+          if (!ptx::mbar_wait(&bars[kSbVFull + s], (g >> 1) & 1, limit)) { ok = false; break; }
+          // the next tile's K, probed where this thread would otherwise wait for P0
+          const bool more = j + 1 < n_tiles || i + 1 < n_my;
+          k_ready = more && ptx::mbar_try_wait(&bars[kSbKFull + (s ^ 1)], ((g + 1) >> 1) & 1);
+          if (!issue_pv(0, g, j)) { ok = false; break; }
+          if (j == n_tiles - 1) ptx::mma_commit(&bars[kSbODone + 0]);
+        }
+      }
+      if (ok && g > 0) {
+        if (issue_pv(1, g - 1, n_tiles - 1))
+          ptx::mma_commit(&bars[kSbODone + 1]);
+        else
+          ok = false;
+      }
+      if (!ok) atomicOr(p.status, kStatusTimeout);
+      // everything issued must complete before TMEM is released
+      ptx::mma_commit(&bars[kSbDrain]);
+      ptx::mbar_wait(&bars[kSbDrain], 0, kDrainNs);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax warpgroups
+    const int wg = warp >> 2;         // 0 or 1
+    const int wq = warp & 3;          // warp within the warpgroup -> TMEM lanes 32*wq..
+    const int r = threadIdx.x & 127;  // query row within the tile
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const uint32_t tS = lane_base + col_s(wg);
+    const uint32_t tO = lane_base + col_o(wg);
+    const float sl2 = p.scale_log2;
+    const uint64_t c2 = ptx::f2_pack(sl2, sl2);
+    uint8_t* ostage = smem + kSmemStage + wg * kSlab;
+    int rag_j[kMaxSegs], rag_v[kMaxSegs];
+    {
+      int first = 0;
+#pragma unroll
+      for (int sg = 0; sg < kMaxSegs; ++sg) {
+        rag_j[sg] = -1;
+        rag_v[sg] = kBN;
+        if (sg < p.n_segs) {
+          const int nt = (p.seg[sg].n_rows + kBN - 1) / kBN;
+          rag_j[sg] = first + nt - 1;
+          rag_v[sg] = p.seg[sg].n_rows - (nt - 1) * kBN;
+          first += nt;
         }
       }
     }
+    FlowStep step;
+    step.sigma = p.sigma;
+    step.renoise = p.sigma_next >= 0.0;
+    step.sigma_next = step.renoise ? p.sigma_next : 0.0;
+    step.one_minus_next = __dsub_rn(1.0, step.sigma_next);
+    // After an expired wait a warp skips all further waits and work but still runs every
+    // named barrier of its warpgroup, so the warpgroup's four warps never part ways there.
+    bool ok = true;
+    int g = 0;
+    for (int i = 0; i < n_my; ++i) {
+      const int u = static_cast<int>(blockIdx.x) + i * G;
+      const int head = u / n_qb;
+      const int row0 = (u - head * n_qb) * (2 * kBM) + wg * kBM;
+      float m_used = -INFINITY;
+      float l = 0.f;
+      float pend = 1.0f;
+      for (int j = 0; j < n_tiles; ++j, ++g) {
+        if (ok) ok = __all_sync(0xffffffffu, ptx::mbar_wait(&bars[kSbSFull + wg], g & 1, limit));
+        if (!ok) continue;
+        ptx::tc_fence_after();
+        int valid = kBN;
+#pragma unroll
+        for (int sg = 0; sg < kMaxSegs; ++sg)
+          if (j == rag_j[sg]) valid = rag_v[sg];
+        if (__any_sync(0xffffffffu, pend != 1.0f)) scale_o(tO, pend);
+        l *= pend;
+        pend = 1.0f;
+        bool stored = false;
+        if (j > 0) {
+          const uint64_t nm2 = ptx::f2_pack(-m_used, -m_used);
+          uint64_t acc[4] = {0, 0, 0, 0};
+          uint32_t pk[kBN / 2];
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t sh[kBN / 2];
+            ptx::tmem_ld64(tS + 64 * hh, sh);
+            if (valid < kBN) {
+#pragma unroll
+              for (int q = 0; q < kBN / 2; ++q)
+                if (64 * hh + q >= valid) sh[q] = 0xff800000u;
+              numerators_half<false>(sh, c2, nm2, pk + 32 * hh, acc);
+            } else {
+              numerators_half<true>(sh, c2, nm2, pk + 32 * hh, acc);
+            }
+          }
+          float rs[4];
+          ptx::f2_unpack(ptx::f2_add(acc[0], acc[1]), rs[0], rs[1]);
+          ptx::f2_unpack(ptx::f2_add(acc[2], acc[3]), rs[2], rs[3]);
+          const float lt = (rs[0] + rs[1]) + (rs[2] + rs[3]);
+          if (!__any_sync(0xffffffffu, !(lt <= kSumSlack))) {
+            l += lt;
+            if (lt > kLazySum) {
+              const float shf = lg2_approx(lt);
+              pend = ptx::ex2(-shf);
+              m_used += shf;
+            }
+            ptx::tmem_st64(tS, pk);
+            stored = true;
+          }
+        }
+        if (!stored) {
+          float m_tile;
+          {
+            uint32_t sr[kBN];
+            ptx::tmem_ld128(tS, sr);
+            if (valid < kBN) {
+#pragma unroll
+              for (int q = 0; q < kBN; ++q)
+                if (q >= valid) sr[q] = 0xff800000u;
+            }
+            float mq[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const uint32_t* t = sr + 32 * c;
+              float m = ptx::fmax3(__uint_as_float(t[0]), __uint_as_float(t[1]), __uint_as_float(t[2]));
+#pragma unroll
+              for (int q = 3; q < 31; q += 2) m = ptx::fmax3(m, __uint_as_float(t[q]), __uint_as_float(t[q + 1]));
+              mq[c] = fmaxf(m, __uint_as_float(t[31]));
+            }
+            m_tile = ptx::fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3])) * sl2;
+          }
+          const bool need = m_tile > m_used + kLazyRescale;
+          float alpha = 1.0f;
+          if (need) {
+            alpha = ptx::ex2(m_used - m_tile);
+            m_used = m_tile;
+          }
+          l *= alpha;
+          if (j > 0 && __any_sync(0xffffffffu, need)) scale_o(tO, alpha);
+          const uint64_t nm2 = ptx::f2_pack(-m_used, -m_used);
+          uint64_t acc[4] = {0, 0, 0, 0};
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t sh[kBN / 2];
+            ptx::tmem_ld64(tS + 64 * hh, sh);
+            if (valid < kBN) {
+#pragma unroll
+              for (int q = 0; q < kBN / 2; ++q)
+                if (64 * hh + q >= valid) sh[q] = 0xff800000u;
+              softmax_half<false>(sh, c2, nm2, tS + 32 * hh, acc);
+            } else {
+              softmax_half<true>(sh, c2, nm2, tS + 32 * hh, acc);
+            }
+          }
+          float rs[4];
+          ptx::f2_unpack(ptx::f2_add(acc[0], acc[1]), rs[0], rs[1]);
+          ptx::f2_unpack(ptx::f2_add(acc[2], acc[3]), rs[2], rs[3]);
+          l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+        }
+        ptx::tmem_st_wait();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&bars[kSbPFull + wg]);
+      }
+      if (ok) ok = __all_sync(0xffffffffu, ptx::mbar_wait(&bars[kSbODone + wg], i & 1, limit));
+      if (ok) ptx::tc_fence_after();
+      // -------------------------------------------------------- epilogue of this unit's tile
+      const int row = row0 + r;
+      const bool live = row < p.Lq;
+      const float inv_l = 1.0f / l;
+      const long long base = (static_cast<long long>(row) * p.H + head) * kHeadDim;
+      const bool store = ok && row0 < p.Lq;  // a tile wholly past Lq writes nothing
+      // the previous unit's second-half store must have read the staging buffer
+      if (r == 0) ptx::bulk_wait_read_all();
+      ptx::named_bar_sync(1 + wg, kBM);
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        if (c == 2) {
+          // first half staged: store it, and wait for its read before the second half
+          ptx::fence_proxy_async_smem();
+          ptx::named_bar_sync(1 + wg, kBM);
+          if (r == 0 && store) {
+            ptx::tma_store_3d(&tm_o, ostage, 0, head, row0);
+            ptx::bulk_commit_group();
+            ptx::bulk_wait_read_all();
+          }
+          ptx::named_bar_sync(1 + wg, kBM);
+        }
+        if (!ok) continue;
+        uint32_t rr[32];
+        ptx::tmem_ld32(tO + 32 * c, rr);
+        uint32_t ob[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+          ob[q] = pack_bf16x2(__uint_as_float(rr[2 * q]) * inv_l, __uint_as_float(rr[2 * q + 1]) * inv_l);
+        uint8_t* orow = ostage + r * 128;
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+          *reinterpret_cast<uint4*>(orow + (((((c & 1) << 2) + v) ^ (r & 7)) << 4)) =
+              make_uint4(ob[4 * v], ob[4 * v + 1], ob[4 * v + 2], ob[4 * v + 3]);
+        if (live && p.flow) {
+          const uint4* xtp = reinterpret_cast<const uint4*>(p.xt + base + 32 * c);
+          const uint4* ep = reinterpret_cast<const uint4*>(p.eps + base + 32 * c);
+          uint4* x0p = reinterpret_cast<uint4*>(p.x0 + base + 32 * c);
+          uint4* xnp = reinterpret_cast<uint4*>(p.xt_next + base + 32 * c);
+          const uint4* cp = reinterpret_cast<const uint4*>(p.v_cond + base + 32 * c);
+          const bool cfg = p.v_cond != nullptr;
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const uint4 xv = __ldg(xtp + v);
+            uint4 ev = make_uint4(0, 0, 0, 0), cv = make_uint4(0, 0, 0, 0);
+            if (step.renoise) ev = __ldg(ep + v);
+            if (cfg) cv = __ldg(cp + v);
+            const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+            const uint32_t ew[4] = {ev.x, ev.y, ev.z, ev.w};
+            const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
+            uint32_t o0[4], o1[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint32_t vw = ob[4 * v + q];
+              uint16_t a0, a1, b0 = 0, b1 = 0;
+              if (cfg) {
+                step.apply_cfg_bits(xw[q], cw[q], vw, ew[q], p.cfg_scale, a0, b0);
+                step.apply_cfg_bits(xw[q] >> 16, cw[q] >> 16, vw >> 16, ew[q] >> 16, p.cfg_scale, a1, b1);
+              } else {
+                step.apply_bits(xw[q], vw, ew[q], a0, b0);
+                step.apply_bits(xw[q] >> 16, vw >> 16, ew[q] >> 16, a1, b1);
+              }
+              o0[q] = static_cast<uint32_t>(a0) | (static_cast<uint32_t>(a1) << 16);
+              o1[q] = static_cast<uint32_t>(b0) | (static_cast<uint32_t>(b1) << 16);
+            }
+            x0p[v] = make_uint4(o0[0], o0[1], o0[2], o0[3]);
+            if (step.renoise) xnp[v] = make_uint4(o1[0], o1[1], o1[2], o1[3]);
+          }
+        }
+      }
+      ptx::fence_proxy_async_smem();
+      ptx::named_bar_sync(1 + wg, kBM);
+      if (r == 0 && store) {
+        ptx::tma_store_3d(&tm_o, ostage, 64, head, row0);
+        ptx::bulk_commit_group();  // read completion is awaited before the buffer is reused
+      }
+    }
+    if (!ok && lane == 0) atomicOr(p.status, kStatusTimeout);
+    if (r == 0) ptx::bulk_wait_read_all();  // the buffer must stay until the last copy has read it
   }
 
   ptx::tc_fence_before();
@@ -615,7 +997,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-// Key streams of at most this many 128-key tiles take the staged-epilogue form.
+// Key streams of at most this many 128-key tiles take the short-stream form.
 constexpr int kShortStreamTiles = 16;
 
 cudaError_t launch_attention(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_vc,
@@ -626,6 +1008,7 @@ cudaError_t launch_attention(const CUtensorMap& tm_q, const CUtensorMap& tm_k, c
   constexpr int kMaxDevices = 64;
   static std::mutex mu;
   static bool configured[kMaxDevices] = {};
+  static int sms[kMaxDevices] = {};
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
@@ -633,20 +1016,24 @@ cudaError_t launch_attention(const CUtensorMap& tm_q, const CUtensorMap& tm_k, c
   {
     std::lock_guard<std::mutex> lock(mu);
     if (!configured[dev]) {
-      err = cudaFuncSetAttribute(chunk_attention_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kSmemBytes);
+      err = cudaFuncSetAttribute(chunk_attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
       if (err == cudaSuccess)
-        err = cudaFuncSetAttribute(chunk_attention_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   kSmemBytes);
+        err = cudaFuncSetAttribute(chunk_attention_short_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   kSmemBytesShort);
+      if (err == cudaSuccess) err = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
       if (err != cudaSuccess) return err;
       configured[dev] = true;
     }
   }
-  dim3 grid((p.Lq + 2 * kBM - 1) / (2 * kBM), p.H);
-  if (p.n_tiles <= kShortStreamTiles)
-    chunk_attention_kernel<true><<<grid, kThreads, kSmemBytes, stream>>>(tm_q, tm_k, tm_vc, tm_vn, tm_o, p);
-  else
-    chunk_attention_kernel<false><<<grid, kThreads, kSmemBytes, stream>>>(tm_q, tm_k, tm_vc, tm_vn, tm_o, p);
+  const int n_qb = (p.Lq + 2 * kBM - 1) / (2 * kBM);
+  if (p.n_tiles <= kShortStreamTiles) {
+    const long long units = static_cast<long long>(n_qb) * p.H;
+    const unsigned grid = static_cast<unsigned>(std::min<long long>(units, sms[dev] > 0 ? sms[dev] : 1));
+    chunk_attention_short_kernel<<<grid, kThreads, kSmemBytesShort, stream>>>(tm_q, tm_k, tm_vc, tm_vn, tm_o, p);
+  } else {
+    dim3 grid(n_qb, p.H);
+    chunk_attention_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_q, tm_k, tm_vc, tm_vn, p);
+  }
   return cudaGetLastError();
 }
 
