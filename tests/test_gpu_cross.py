@@ -163,3 +163,32 @@ def test_cross_longest_text_context():
         h.set_text_kv(0, k2, k2)
     assert h.poll_device_status() == rkv.OK
     h.close()
+
+
+def test_cross_timeout_with_several_units_per_cta():
+    """More query blocks than SMs (4 heads x 40 blocks of 256 queries = 160 units), so CTAs of
+    the persistent short-stream kernel run two units each. A 1 ns wait cap makes waits expire
+    at arbitrary points of that walk, possibly in some warps of a warpgroup and not in others:
+    the call must come back with RKV_ERR_TIMEOUT, and the next call with the normal cap must
+    match the oracle."""
+    H, n_text, n_q = 4, 512, 40 * 256
+    h = rkv.RollingKV(1, H, 128, 4, 6, 2, OracleLayer.ABSOLUTE)
+    kt, ktb = _pair(H, n_text, synth.stream_key(0, 76, 1))
+    vt, vtb = _pair(H, n_text, synth.stream_key(0, 76, 2))
+    h.set_text_kv(0, kt, vt)
+    q, qb = _pair(H, n_q, synth.stream_key(0, 76, 3))
+    out = torch.zeros_like(q)
+    h.set_wait_limit(1)
+    for _ in range(3):
+        h.cross_attention(0, q, out)
+        assert h.poll_device_status() == rkv.ERR_TIMEOUT
+    h.set_wait_limit(2_000_000_000)
+    h.cross_attention(0, q, out)
+    assert h.poll_device_status() == rkv.OK
+    orc = _oracle(H)
+    orc.set_text_kv(ktb, vtb)
+    rows = np.arange(0, n_q, 37)
+    got = to_bits(out)[rows]
+    want = orc.cross_attention(qb[rows])
+    assert_close(got, want, "after timeouts")
+    h.close()
