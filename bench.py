@@ -395,6 +395,8 @@ def measure_workload(args, name, headline):
         h.close()
         del pool, outs, x0, xn
         torch.cuda.empty_cache()
+        traffic, traffic_src, traffic_alg = profiled_traffic(name)
+        attn.update(traffic=traffic, traffic_source=traffic_src, traffic_algorithmic_bytes=traffic_alg)
         return {"workload": cfg["workload"], "value": value, "unit": UNIT, "steps": args.steps,
                 "ms_per_step": ms / args.steps, "queries_per_call": Lq, "keys_per_call": W * T,
                 "attention": attn, "hbm_kernels": hbm, "clocks": clk}
