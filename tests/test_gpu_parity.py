@@ -15,7 +15,7 @@ import pytest
 import synth
 from oracle import bf16, flow as oflow
 from oracle.layer import OracleLayer
-from rollout import Config, Rollout, assert_close, cache_logical_bits, dev_tensor, host_bits, to_bits
+from rollout import Config, Rollout, assert_close, cache_logical_bits, dev_tensor, host_bits, sample_rows, to_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -602,3 +602,35 @@ def _copy_on_stream(t):
     c = torch.empty_like(t)
     c.copy_(t, non_blocking=True)
     return c
+
+
+def test_fused_flow_with_more_units_than_sms():
+    """A short key stream (1560 keys = 13 tiles: the persistent short-stream kernel) with 40
+    heads x 7 query blocks = 280 units, so CTAs walk two units each, with the fused x0 /
+    renoise epilogue: x0 and xt' bit-exact against the oracle's step on the stored output, the
+    output on sampled rows of sampled heads within the attention tolerance, through three
+    chunks (the window rolls)."""
+    cfg = Config("units", 17, H=40, grid_h=30, grid_w=52, C=1, W=1, S=0, rope_mode=ABS, chunks=1)
+    h = rkv.RollingKV(1, cfg.H, 128, cfg.T, cfg.W, cfg.S, cfg.rope_mode)
+    h.set_rope_grid(cfg.grid_h, cfg.grid_w)
+    orc = OracleLayer(cfg.H, 128, cfg.T, cfg.grid_h, cfg.grid_w, cfg.W, cfg.S, cfg.rope_mode)
+    Lq, n = cfg.Lq, cfg.Lq * cfg.H * 128
+    rows = sample_rows(Lq, n=48, seed=5)
+    heads = [0, 17, 39]
+    for chunk in range(3):
+        q, k, v = (dev_tensor(torch, cfg, 0, chunk, 0, t, Lq) for t in ("q", "k", "v"))
+        xt = _dev_bits(synth.stream_key(0, 17, chunk, 1), n)
+        eps = _dev_bits(synth.stream_key(0, 17, chunk, 2), n)
+        out = torch.empty((Lq, cfg.H, 128), dtype=torch.bfloat16, device="cuda")
+        x0 = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+        xn = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+        h.chunk_attention(0, q, k, v, out, cfg.C, chunk, True,
+                          flow=dict(xt=xt, eps=eps, sigma=0.75, sigma_next=0.5, x0_out=x0, xt_next_out=xn))
+        torch.cuda.synchronize()
+        assert h.poll_device_status() == rkv.OK
+        rx0, rxn = oflow.x0_renoise_bf16(to_bits(xt), to_bits(out).reshape(-1), to_bits(eps), 0.75, 0.5)
+        assert np.array_equal(to_bits(x0), rx0) and np.array_equal(to_bits(xn), rxn)
+        qb, kb, vb = (to_bits(t) for t in (q, k, v))
+        ref = orc.chunk_attention(qb, kb, vb, cfg.C, chunk, True, rows=rows, heads=heads)
+        assert_close(to_bits(out)[rows][:, heads], ref, f"chunk {chunk}")
+    h.close()
