@@ -11,9 +11,14 @@
 // only masking is of the ragged last tile of each segment.
 //
 // Queries and keys arrive already rotated (RoPE applied by the frame-run kernel on
-// their way into the head-major staging / rotated-K ring), V raw. The same kernel serves
+// their way into the head-major staging / rotated-K ring), V raw. The same kernels serve
 // the cross-attention over the cached text K/V: one key segment, queries read token-major
 // straight from the caller's buffer, no rotation.
+//
+// Two kernels: chunk_attention_kernel (one CTA per unit of one head x 256 query rows) for
+// long key streams, and chunk_attention_short_kernel, a persistent form for key streams of
+// at most kShortStreamTiles tiles (described at its definition). Both share the structure
+// and the softmax below.
 //
 // Structure of one CTA (one head, 256 query rows = two 128-row tiles Q0, Q1):
 //   warps 0-3  softmax for Q0 (one thread per query row = TMEM lane)
@@ -224,6 +229,178 @@ __device__ __forceinline__ void scale_o(uint32_t tO, float f) {
   }
 }
 
+// The x0 / renoise step (and the guidance combine when v_cond is set; this launch is then the
+// unconditional branch, its output u) on 32 consecutive elements of this thread's row:
+// ob holds the attention output of those elements as stored (bf16 pairs), off their index
+// in the latent [Lq, H * d].
+__device__ __forceinline__ void flow_epilogue32(const AttnParams& p, const FlowStep& step, long long off,
+                                                const uint32_t (&ob)[16]) {
+  const uint4* xtp = reinterpret_cast<const uint4*>(p.xt + off);
+  const uint4* ep = reinterpret_cast<const uint4*>(p.eps + off);
+  uint4* x0p = reinterpret_cast<uint4*>(p.x0 + off);
+  uint4* xnp = reinterpret_cast<uint4*>(p.xt_next + off);
+  const uint4* cp = reinterpret_cast<const uint4*>(p.v_cond + off);
+  const bool cfg = p.v_cond != nullptr;
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    const uint4 xv = __ldg(xtp + v);
+    uint4 ev = make_uint4(0, 0, 0, 0), cv = make_uint4(0, 0, 0, 0);
+    if (step.renoise) ev = __ldg(ep + v);
+    if (cfg) cv = __ldg(cp + v);
+    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+    const uint32_t ew[4] = {ev.x, ev.y, ev.z, ev.w};
+    const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
+    uint32_t o0[4], o1[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t vw = ob[4 * v + q];
+      uint16_t a0, a1, b0 = 0, b1 = 0;
+      if (cfg) {
+        step.apply_cfg_bits(xw[q], cw[q], vw, ew[q], p.cfg_scale, a0, b0);
+        step.apply_cfg_bits(xw[q] >> 16, cw[q] >> 16, vw >> 16, ew[q] >> 16, p.cfg_scale, a1, b1);
+      } else {
+        step.apply_bits(xw[q], vw, ew[q], a0, b0);
+        step.apply_bits(xw[q] >> 16, vw >> 16, ew[q] >> 16, a1, b1);
+      }
+      o0[q] = static_cast<uint32_t>(a0) | (static_cast<uint32_t>(a1) << 16);
+      o1[q] = static_cast<uint32_t>(b0) | (static_cast<uint32_t>(b1) << 16);
+    }
+    x0p[v] = make_uint4(o0[0], o0[1], o0[2], o0[3]);
+    if (step.renoise) xnp[v] = make_uint4(o1[0], o1[1], o1[2], o1[3]);
+  }
+}
+
+// The ragged last tile of each key segment: its index in the key stream and its number of
+// valid keys (-1 and kBN for absent segments).
+__device__ __forceinline__ void ragged_tiles(const AttnParams& p, int (&rag_j)[kMaxSegs], int (&rag_v)[kMaxSegs]) {
+  int first = 0;
+#pragma unroll
+  for (int sg = 0; sg < kMaxSegs; ++sg) {
+    rag_j[sg] = -1;
+    rag_v[sg] = kBN;
+    if (sg < p.n_segs) {
+      const int nt = (p.seg[sg].n_rows + kBN - 1) / kBN;
+      rag_j[sg] = first + nt - 1;
+      rag_v[sg] = p.seg[sg].n_rows - (nt - 1) * kBN;
+      first += nt;
+    }
+  }
+}
+
+// valid keys of key tile j (kBN unless it is a segment's ragged last tile)
+__device__ __forceinline__ int tile_valid(int j, const int (&rag_j)[kMaxSegs], const int (&rag_v)[kMaxSegs]) {
+  int valid = kBN;
+#pragma unroll
+  for (int sg = 0; sg < kMaxSegs; ++sg)
+    if (j == rag_j[sg]) valid = rag_v[sg];
+  return valid;
+}
+
+// One key tile of this thread's query row: apply a pending change of reference to O and l,
+// form the numerators of S(j) (one pass against the running reference, or the exact path
+// on the first tile and after a score far above the reference) and leave P over S in TMEM.
+// m_used: reference of the numerators in log2 units (p = 2^(s * sl2 - m_used)); l: row sum
+// of the numerators in that reference's scale; pend: change of reference decided on this
+// tile, applied at the next (when PV(j) has completed). The caller waits for the TMEM
+// stores and signals P.
+__device__ __forceinline__ void softmax_tile(int j, int valid, uint32_t tS, uint32_t tO, float sl2, uint64_t c2,
+                                             float& m_used, float& l, float& pend) {
+  // S(j) complete implies PV(j-1) complete: O now holds every product in the previous
+  // reference's scale, so a pending change applies to O and l together
+  if (__any_sync(0xffffffffu, pend != 1.0f)) scale_o(tO, pend);
+  l *= pend;
+  pend = 1.0f;
+  bool stored = false;
+  if (j > 0) {
+    // one pass against the running reference
+    const uint64_t nm2 = ptx::f2_pack(-m_used, -m_used);
+    uint64_t acc[4] = {0, 0, 0, 0};
+    uint32_t pk[kBN / 2];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      uint32_t sh[kBN / 2];
+      ptx::tmem_ld64(tS + 64 * hh, sh);
+      if (valid < kBN) {
+#pragma unroll
+        for (int i = 0; i < kBN / 2; ++i)
+          if (64 * hh + i >= valid) sh[i] = 0xff800000u;
+        numerators_half<false>(sh, c2, nm2, pk + 32 * hh, acc);
+      } else {
+        numerators_half<true>(sh, c2, nm2, pk + 32 * hh, acc);
+      }
+    }
+    float rs[4];
+    ptx::f2_unpack(ptx::f2_add(acc[0], acc[1]), rs[0], rs[1]);
+    ptx::f2_unpack(ptx::f2_add(acc[2], acc[3]), rs[2], rs[3]);
+    const float lt = (rs[0] + rs[1]) + (rs[2] + rs[3]);
+    // the tile's numerator sum bounds its largest numerator: 2^max <= lt <= 128 * 2^max.
+    // A sum above 2^64 (or not a number) sends the warp to the exact path below.
+    if (!__any_sync(0xffffffffu, !(lt <= kSumSlack))) {
+      l += lt;
+      if (lt > kLazySum) {  // move the reference up by log2(lt) from the next tile on
+        const float sh = lg2_approx(lt);
+        pend = ptx::ex2(-sh);
+        m_used += sh;
+      }
+      ptx::tmem_st64(tS, pk);
+      stored = true;
+    }
+  }
+  if (!stored) {
+    // exact path (the first tile, or a score far above the reference): the row maximum
+    // first, then the numerators
+    float m_tile;
+    {
+      uint32_t sr[kBN];
+      ptx::tmem_ld128(tS, sr);
+      if (valid < kBN) {
+#pragma unroll
+        for (int i = 0; i < kBN; ++i)
+          if (i >= valid) sr[i] = 0xff800000u;
+      }
+      float mq[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const uint32_t* t = sr + 32 * c;
+        float m = ptx::fmax3(__uint_as_float(t[0]), __uint_as_float(t[1]), __uint_as_float(t[2]));
+#pragma unroll
+        for (int i = 3; i < 31; i += 2) m = ptx::fmax3(m, __uint_as_float(t[i]), __uint_as_float(t[i + 1]));
+        mq[c] = fmaxf(m, __uint_as_float(t[31]));
+      }
+      m_tile = ptx::fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3])) * sl2;
+    }
+    const bool need = m_tile > m_used + kLazyRescale;
+    float alpha = 1.0f;
+    if (need) {
+      alpha = ptx::ex2(m_used - m_tile);
+      m_used = m_tile;
+    }
+    l *= alpha;
+    if (j > 0 && __any_sync(0xffffffffu, need)) scale_o(tO, alpha);
+    const uint64_t nm2 = ptx::f2_pack(-m_used, -m_used);
+    uint64_t acc[4] = {0, 0, 0, 0};
+    // reload 64 columns at a time; P of the first half overwrites S columns 0..31,
+    // already read, the second half's loads touch columns 64..127 only
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      uint32_t sh[kBN / 2];
+      ptx::tmem_ld64(tS + 64 * hh, sh);
+      if (valid < kBN) {
+#pragma unroll
+        for (int i = 0; i < kBN / 2; ++i)
+          if (64 * hh + i >= valid) sh[i] = 0xff800000u;
+        softmax_half<false>(sh, c2, nm2, tS + 32 * hh, acc);
+      } else {
+        softmax_half<true>(sh, c2, nm2, tS + 32 * hh, acc);
+      }
+    }
+    float rs[4];
+    ptx::f2_unpack(ptx::f2_add(acc[0], acc[1]), rs[0], rs[1]);
+    ptx::f2_unpack(ptx::f2_add(acc[2], acc[3]), rs[2], rs[3]);
+    l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                            const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_vn,
@@ -373,124 +550,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     float pend = 1.0f;         // change of reference decided on the previous tile, not yet applied
     // the ragged last tile of each key segment: its index in the stream and its valid keys
     int rag_j[kMaxSegs], rag_v[kMaxSegs];
-    {
-      int first = 0;
-#pragma unroll
-      for (int sg = 0; sg < kMaxSegs; ++sg) {
-        rag_j[sg] = -1;
-        rag_v[sg] = kBN;
-        if (sg < p.n_segs) {
-          const int nt = (p.seg[sg].n_rows + kBN - 1) / kBN;
-          rag_j[sg] = first + nt - 1;
-          rag_v[sg] = p.seg[sg].n_rows - (nt - 1) * kBN;
-          first += nt;
-        }
-      }
-    }
+    ragged_tiles(p, rag_j, rag_v);
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
       ok = ptx::mbar_wait(&bars[kBarSFull + wg], j & 1, limit);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       ptx::tc_fence_after();
-      int valid = kBN;
-#pragma unroll
-      for (int sg = 0; sg < kMaxSegs; ++sg)
-        if (j == rag_j[sg]) valid = rag_v[sg];
-      // S(j) complete implies PV(j-1) complete: O now holds every product in the previous
-      // reference's scale, so a pending change applies to O and l together
-      if (__any_sync(0xffffffffu, pend != 1.0f)) scale_o(tO, pend);
-      l *= pend;
-      pend = 1.0f;
-      bool stored = false;
-      if (j > 0) {
-        // one pass against the running reference
-        const uint64_t nm2 = ptx::f2_pack(-m_used, -m_used);
-        uint64_t acc[4] = {0, 0, 0, 0};
-        uint32_t pk[kBN / 2];
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          uint32_t sh[kBN / 2];
-          ptx::tmem_ld64(tS + 64 * hh, sh);
-          if (valid < kBN) {
-#pragma unroll
-            for (int i = 0; i < kBN / 2; ++i)
-              if (64 * hh + i >= valid) sh[i] = 0xff800000u;
-            numerators_half<false>(sh, c2, nm2, pk + 32 * hh, acc);
-          } else {
-            numerators_half<true>(sh, c2, nm2, pk + 32 * hh, acc);
-          }
-        }
-        float rs[4];
-        ptx::f2_unpack(ptx::f2_add(acc[0], acc[1]), rs[0], rs[1]);
-        ptx::f2_unpack(ptx::f2_add(acc[2], acc[3]), rs[2], rs[3]);
-        const float lt = (rs[0] + rs[1]) + (rs[2] + rs[3]);
-        // the tile's numerator sum bounds its largest numerator: 2^max <= lt <= 128 * 2^max.
-        // A sum above 2^64 (or not a number) sends the warp to the exact path below.
-        if (!__any_sync(0xffffffffu, !(lt <= kSumSlack))) {
-          l += lt;
-          if (lt > kLazySum) {  // move the reference up by log2(lt) from the next tile on
-            const float sh = lg2_approx(lt);
-            pend = ptx::ex2(-sh);
-            m_used += sh;
-          }
-          ptx::tmem_st64(tS, pk);
-          stored = true;
-        }
-      }
-      if (!stored) {
-        // exact path (the first tile, or a score far above the reference): the row maximum
-        // first, then the numerators
-        float m_tile;
-        {
-          uint32_t sr[kBN];
-          ptx::tmem_ld128(tS, sr);
-          if (valid < kBN) {
-#pragma unroll
-            for (int i = 0; i < kBN; ++i)
-              if (i >= valid) sr[i] = 0xff800000u;
-          }
-          float mq[4];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const uint32_t* t = sr + 32 * c;
-            float m = ptx::fmax3(__uint_as_float(t[0]), __uint_as_float(t[1]), __uint_as_float(t[2]));
-#pragma unroll
-            for (int i = 3; i < 31; i += 2) m = ptx::fmax3(m, __uint_as_float(t[i]), __uint_as_float(t[i + 1]));
-            mq[c] = fmaxf(m, __uint_as_float(t[31]));
-          }
-          m_tile = ptx::fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3])) * sl2;
-        }
-        const bool need = m_tile > m_used + kLazyRescale;
-        float alpha = 1.0f;
-        if (need) {
-          alpha = ptx::ex2(m_used - m_tile);
-          m_used = m_tile;
-        }
-        l *= alpha;
-        if (j > 0 && __any_sync(0xffffffffu, need)) scale_o(tO, alpha);
-        const uint64_t nm2 = ptx::f2_pack(-m_used, -m_used);
-        uint64_t acc[4] = {0, 0, 0, 0};
-        // reload 64 columns at a time; P of the first half overwrites S columns 0..31,
-        // already read, the second half's loads touch columns 64..127 only
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          uint32_t sh[kBN / 2];
-          ptx::tmem_ld64(tS + 64 * hh, sh);
-          if (valid < kBN) {
-#pragma unroll
-            for (int i = 0; i < kBN / 2; ++i)
-              if (64 * hh + i >= valid) sh[i] = 0xff800000u;
-            softmax_half<false>(sh, c2, nm2, tS + 32 * hh, acc);
-          } else {
-            softmax_half<true>(sh, c2, nm2, tS + 32 * hh, acc);
-          }
-        }
-        float rs[4];
-        ptx::f2_unpack(ptx::f2_add(acc[0], acc[1]), rs[0], rs[1]);
-        ptx::f2_unpack(ptx::f2_add(acc[2], acc[3]), rs[2], rs[3]);
-        l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
-      }
+      const int valid = tile_valid(j, rag_j, rag_v);
+      softmax_tile(j, valid, tS, tO, sl2, c2, m_used, l, pend);
       ptx::tmem_st_wait();
       ptx::tc_fence_before();
       ptx::mbar_arrive(&bars[kBarPFull + wg]);
@@ -524,42 +592,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint4* dst = reinterpret_cast<uint4*>(p.out + base + 32 * c);
 #pragma unroll
           for (int v = 0; v < 4; ++v) dst[v] = make_uint4(ob[4 * v], ob[4 * v + 1], ob[4 * v + 2], ob[4 * v + 3]);
-          if (p.flow) {
-            const uint4* xtp = reinterpret_cast<const uint4*>(p.xt + base + 32 * c);
-            const uint4* ep = reinterpret_cast<const uint4*>(p.eps + base + 32 * c);
-            uint4* x0p = reinterpret_cast<uint4*>(p.x0 + base + 32 * c);
-            uint4* xnp = reinterpret_cast<uint4*>(p.xt_next + base + 32 * c);
-            const uint4* cp = reinterpret_cast<const uint4*>(p.v_cond + base + 32 * c);
-            const bool cfg = p.v_cond != nullptr;
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              const uint4 xv = __ldg(xtp + v);
-              uint4 ev = make_uint4(0, 0, 0, 0), cv = make_uint4(0, 0, 0, 0);
-              if (step.renoise) ev = __ldg(ep + v);
-              if (cfg) cv = __ldg(cp + v);
-              const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-              const uint32_t ew[4] = {ev.x, ev.y, ev.z, ev.w};
-              const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
-              uint32_t o0[4], o1[4];
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const uint32_t vw = ob[4 * v + q];
-                uint16_t a0, a1, b0 = 0, b1 = 0;
-                if (cfg) {
-                  // this launch is the unconditional branch: its output is u
-                  step.apply_cfg_bits(xw[q], cw[q], vw, ew[q], p.cfg_scale, a0, b0);
-                  step.apply_cfg_bits(xw[q] >> 16, cw[q] >> 16, vw >> 16, ew[q] >> 16, p.cfg_scale, a1, b1);
-                } else {
-                  step.apply_bits(xw[q], vw, ew[q], a0, b0);
-                  step.apply_bits(xw[q] >> 16, vw >> 16, ew[q] >> 16, a1, b1);
-                }
-                o0[q] = static_cast<uint32_t>(a0) | (static_cast<uint32_t>(a1) << 16);
-                o1[q] = static_cast<uint32_t>(b0) | (static_cast<uint32_t>(b1) << 16);
-              }
-              x0p[v] = make_uint4(o0[0], o0[1], o0[2], o0[3]);
-              if (step.renoise) xnp[v] = make_uint4(o1[0], o1[1], o1[2], o1[3]);
-            }
-          }
+          if (p.flow) flow_epilogue32(p, step, base + 32 * c, ob);
         }
       }
     }
@@ -779,20 +812,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t c2 = ptx::f2_pack(sl2, sl2);
     uint8_t* ostage = smem + kSmemStage + wg * kSlab;
     int rag_j[kMaxSegs], rag_v[kMaxSegs];
-    {
-      int first = 0;
-#pragma unroll
-      for (int sg = 0; sg < kMaxSegs; ++sg) {
-        rag_j[sg] = -1;
-        rag_v[sg] = kBN;
-        if (sg < p.n_segs) {
-          const int nt = (p.seg[sg].n_rows + kBN - 1) / kBN;
-          rag_j[sg] = first + nt - 1;
-          rag_v[sg] = p.seg[sg].n_rows - (nt - 1) * kBN;
-          first += nt;
-        }
-      }
-    }
+    ragged_tiles(p, rag_j, rag_v);
     FlowStep step;
     step.sigma = p.sigma;
     step.renoise = p.sigma_next >= 0.0;
@@ -813,95 +833,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) ok = __all_sync(0xffffffffu, ptx::mbar_wait(&bars[kSbSFull + wg], g & 1, limit));
         if (!ok) continue;
         ptx::tc_fence_after();
-        int valid = kBN;
-#pragma unroll
-        for (int sg = 0; sg < kMaxSegs; ++sg)
-          if (j == rag_j[sg]) valid = rag_v[sg];
-        if (__any_sync(0xffffffffu, pend != 1.0f)) scale_o(tO, pend);
-        l *= pend;
-        pend = 1.0f;
-        bool stored = false;
-        if (j > 0) {
-          const uint64_t nm2 = ptx::f2_pack(-m_used, -m_used);
-          uint64_t acc[4] = {0, 0, 0, 0};
-          uint32_t pk[kBN / 2];
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            uint32_t sh[kBN / 2];
-            ptx::tmem_ld64(tS + 64 * hh, sh);
-            if (valid < kBN) {
-#pragma unroll
-              for (int q = 0; q < kBN / 2; ++q)
-                if (64 * hh + q >= valid) sh[q] = 0xff800000u;
-              numerators_half<false>(sh, c2, nm2, pk + 32 * hh, acc);
-            } else {
-              numerators_half<true>(sh, c2, nm2, pk + 32 * hh, acc);
-            }
-          }
-          float rs[4];
-          ptx::f2_unpack(ptx::f2_add(acc[0], acc[1]), rs[0], rs[1]);
-          ptx::f2_unpack(ptx::f2_add(acc[2], acc[3]), rs[2], rs[3]);
-          const float lt = (rs[0] + rs[1]) + (rs[2] + rs[3]);
-          if (!__any_sync(0xffffffffu, !(lt <= kSumSlack))) {
-            l += lt;
-            if (lt > kLazySum) {
-              const float shf = lg2_approx(lt);
-              pend = ptx::ex2(-shf);
-              m_used += shf;
-            }
-            ptx::tmem_st64(tS, pk);
-            stored = true;
-          }
-        }
-        if (!stored) {
-          float m_tile;
-          {
-            uint32_t sr[kBN];
-            ptx::tmem_ld128(tS, sr);
-            if (valid < kBN) {
-#pragma unroll
-              for (int q = 0; q < kBN; ++q)
-                if (q >= valid) sr[q] = 0xff800000u;
-            }
-            float mq[4];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const uint32_t* t = sr + 32 * c;
-              float m = ptx::fmax3(__uint_as_float(t[0]), __uint_as_float(t[1]), __uint_as_float(t[2]));
-#pragma unroll
-              for (int q = 3; q < 31; q += 2) m = ptx::fmax3(m, __uint_as_float(t[q]), __uint_as_float(t[q + 1]));
-              mq[c] = fmaxf(m, __uint_as_float(t[31]));
-            }
-            m_tile = ptx::fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3])) * sl2;
-          }
-          const bool need = m_tile > m_used + kLazyRescale;
-          float alpha = 1.0f;
-          if (need) {
-            alpha = ptx::ex2(m_used - m_tile);
-            m_used = m_tile;
-          }
-          l *= alpha;
-          if (j > 0 && __any_sync(0xffffffffu, need)) scale_o(tO, alpha);
-          const uint64_t nm2 = ptx::f2_pack(-m_used, -m_used);
-          uint64_t acc[4] = {0, 0, 0, 0};
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            uint32_t sh[kBN / 2];
-            ptx::tmem_ld64(tS + 64 * hh, sh);
-            if (valid < kBN) {
-#pragma unroll
-              for (int q = 0; q < kBN / 2; ++q)
-                if (64 * hh + q >= valid) sh[q] = 0xff800000u;
-              softmax_half<false>(sh, c2, nm2, tS + 32 * hh, acc);
-            } else {
-              softmax_half<true>(sh, c2, nm2, tS + 32 * hh, acc);
-            }
-          }
-          float rs[4];
-          ptx::f2_unpack(ptx::f2_add(acc[0], acc[1]), rs[0], rs[1]);
-          ptx::f2_unpack(ptx::f2_add(acc[2], acc[3]), rs[2], rs[3]);
-          l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
-        }
+        const int valid = tile_valid(j, rag_j, rag_v);
+        softmax_tile(j, valid, tS, tO, sl2, c2, m_used, l, pend);
         ptx::tmem_st_wait();
         ptx::tc_fence_before();
         ptx::mbar_arrive(&bars[kSbPFull + wg]);
@@ -942,41 +875,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int v = 0; v < 4; ++v)
           *reinterpret_cast<uint4*>(orow + (((((c & 1) << 2) + v) ^ (r & 7)) << 4)) =
               make_uint4(ob[4 * v], ob[4 * v + 1], ob[4 * v + 2], ob[4 * v + 3]);
-        if (live && p.flow) {
-          const uint4* xtp = reinterpret_cast<const uint4*>(p.xt + base + 32 * c);
-          const uint4* ep = reinterpret_cast<const uint4*>(p.eps + base + 32 * c);
-          uint4* x0p = reinterpret_cast<uint4*>(p.x0 + base + 32 * c);
-          uint4* xnp = reinterpret_cast<uint4*>(p.xt_next + base + 32 * c);
-          const uint4* cp = reinterpret_cast<const uint4*>(p.v_cond + base + 32 * c);
-          const bool cfg = p.v_cond != nullptr;
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const uint4 xv = __ldg(xtp + v);
-            uint4 ev = make_uint4(0, 0, 0, 0), cv = make_uint4(0, 0, 0, 0);
-            if (step.renoise) ev = __ldg(ep + v);
-            if (cfg) cv = __ldg(cp + v);
-            const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-            const uint32_t ew[4] = {ev.x, ev.y, ev.z, ev.w};
-            const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
-            uint32_t o0[4], o1[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const uint32_t vw = ob[4 * v + q];
-              uint16_t a0, a1, b0 = 0, b1 = 0;
-              if (cfg) {
-                step.apply_cfg_bits(xw[q], cw[q], vw, ew[q], p.cfg_scale, a0, b0);
-                step.apply_cfg_bits(xw[q] >> 16, cw[q] >> 16, vw >> 16, ew[q] >> 16, p.cfg_scale, a1, b1);
-              } else {
-                step.apply_bits(xw[q], vw, ew[q], a0, b0);
-                step.apply_bits(xw[q] >> 16, vw >> 16, ew[q] >> 16, a1, b1);
-              }
-              o0[q] = static_cast<uint32_t>(a0) | (static_cast<uint32_t>(a1) << 16);
-              o1[q] = static_cast<uint32_t>(b0) | (static_cast<uint32_t>(b1) << 16);
-            }
-            x0p[v] = make_uint4(o0[0], o0[1], o0[2], o0[3]);
-            if (step.renoise) xnp[v] = make_uint4(o1[0], o1[1], o1[2], o1[3]);
-          }
-        }
+        if (live && p.flow) flow_epilogue32(p, step, base + 32 * c, ob);
       }
       ptx::fence_proxy_async_smem();
       ptx::named_bar_sync(1 + wg, kBM);
