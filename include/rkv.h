@@ -22,8 +22,10 @@
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *    stream). Every device launch is asynchronous on that stream; host state
  *    (frames committed, slot map) advances when the call is enqueued.
- *  - Calls on one handle must be issued from one host thread and, for a given
- *    layer, be ordered on one stream (the per-layer scratch is reused).
+ *  - Calls on one handle must be issued from one host thread and be ordered on
+ *    one stream (the per-layer scratch and the handle's scratch for the split
+ *    last wave of long attention launches are reused); separate handles may run
+ *    on separate streams concurrently.
  *  - Return value: RKV_OK or one of the RKV_ERR_* codes below. Argument,
  *    order and capacity errors are detected on the host before anything is
  *    launched; then no state changes.

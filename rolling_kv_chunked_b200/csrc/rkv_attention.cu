@@ -412,8 +412,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int head = blockIdx.y;
-  const int m0 = blockIdx.x * (2 * kBM);
+  // unit u = head * query blocks + block; CTAs from split_first on take half a unit's keys
+  const int n_qb = (p.Lq + 2 * kBM - 1) / (2 * kBM);
+  const int b = static_cast<int>(blockIdx.x);
+  const int half = b >= p.split_first ? (b - p.split_first) & 1 : -1;
+  const int u = half < 0 ? b : p.split_first + ((b - p.split_first) >> 1);
+  const int head = u / n_qb;
+  const int m0 = (u - head * n_qb) * (2 * kBM);
+  const int j0 = half == 1 ? p.split_tiles : 0;  // first key tile of this CTA in the stream
+  const int n_tiles = half < 0 ? p.n_tiles : (half == 0 ? p.split_tiles : p.n_tiles - p.split_tiles);
   const unsigned long long limit = p.wait_limit_ns;
 
   if (threadIdx.x == 0) {
@@ -438,7 +445,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int n_tiles = p.n_tiles;
 
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
@@ -459,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < n_tiles; ++j) {
         const int s = j & 1;
         int src, krow, vrow, valid;
-        tile_of(p, j, src, krow, vrow, valid);
+        tile_of(p, j0 + j, src, krow, vrow, valid);
         if (j >= 2 && !ptx::mbar_wait(&bars[kBarKEmpty + s], ((j - 2) >> 1) & 1, limit)) { ok = false; break; }
         ptx::mbar_arrive_expect_tx(&bars[kBarKFull + s], kTile);
         for (int c = 0; c < 2; ++c)
@@ -557,7 +563,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       ptx::tc_fence_after();
-      const int valid = tile_valid(j, rag_j, rag_v);
+      const int valid = tile_valid(j0 + j, rag_j, rag_v);
       softmax_tile(j, valid, tS, tO, sl2, c2, m_used, l, pend);
       ptx::tmem_st_wait();
       ptx::tc_fence_before();
@@ -569,6 +575,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (!ok) {
       if (lane == 0) atomicOr(p.status, kStatusTimeout);
+    } else if (half >= 0) {
+      // half of a split unit: the unnormalised O row and its sum in the scale of the current
+      // reference (a change decided on the last tile applied here), and the reference, for
+      // the combine launch that follows
+      ptx::tc_fence_after();
+      float* po = p.part + (static_cast<long long>(b - p.split_first) * (2 * kBM) + wg * kBM + r) * kPartRow;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t rr[32];
+        ptx::tmem_ld32(tO + 32 * c, rr);
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+          reinterpret_cast<float4*>(po + 32 * c)[v] =
+              make_float4(__uint_as_float(rr[4 * v]) * pend, __uint_as_float(rr[4 * v + 1]) * pend,
+                          __uint_as_float(rr[4 * v + 2]) * pend, __uint_as_float(rr[4 * v + 3]) * pend);
+      }
+      reinterpret_cast<float4*>(po + 128)[0] = make_float4(m_used, l * pend, 0.f, 0.f);
     } else {
       ptx::tc_fence_after();
       const int row = m0 + wg * kBM + r;
@@ -894,10 +917,73 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 9) ptx::tmem_dealloc(tmem, 512);
 }
 
+
+// The combine of a key-split unit (the last, partial wave of a long stream run as twice as
+// many CTAs over half the keys each): one warp per query row, lane l owning columns
+// 4l .. 4l+3. With the halves' references m_a, m_b and sums l_a, l_b (each half's O and sum
+// in the scale of its own reference), m = max(m_a, m_b) and
+//   O = (O_a 2^(m_a - m) + O_b 2^(m_b - m)) / (l_a 2^(m_a - m) + l_b 2^(m_b - m)),
+// rounded to bf16 (nearest even) and stored token-major; the fused x0 / renoise step (and the
+// guidance combine) then runs on the stored values, as in the attention kernels' epilogue.
+__global__ void __launch_bounds__(256) attention_combine_kernel(const __grid_constant__ AttnParams p) {
+  const int n_qb = (p.Lq + 2 * kBM - 1) / (2 * kBM);
+  const long long gw = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long n_split = static_cast<long long>(n_qb) * p.H - p.split_first;
+  if (gw >= n_split * (2 * kBM)) return;
+  const int t = static_cast<int>(gw / (2 * kBM));
+  const int rr = static_cast<int>(gw - static_cast<long long>(t) * (2 * kBM));
+  const int u = p.split_first + t;
+  const int head = u / n_qb;
+  const int row = (u - head * n_qb) * (2 * kBM) + rr;
+  if (row >= p.Lq) return;
+  const float* pa = p.part + (static_cast<long long>(2 * t) * (2 * kBM) + rr) * kPartRow;
+  const float* pb = pa + static_cast<long long>(2 * kBM) * kPartRow;
+  const float ma = pa[128], la = pa[129], mb = pb[128], lb = pb[129];
+  const float m = fmaxf(ma, mb);
+  const float fa = exp2f(ma - m), fb = exp2f(mb - m);
+  const float inv = 1.0f / (la * fa + lb * fb);
+  const float4 oa = reinterpret_cast<const float4*>(pa)[lane];
+  const float4 ob = reinterpret_cast<const float4*>(pb)[lane];
+  const uint32_t w0 = pack_bf16x2((oa.x * fa + ob.x * fb) * inv, (oa.y * fa + ob.y * fb) * inv);
+  const uint32_t w1 = pack_bf16x2((oa.z * fa + ob.z * fb) * inv, (oa.w * fa + ob.w * fb) * inv);
+  const long long off = (static_cast<long long>(row) * p.H + head) * kHeadDim + 4 * lane;
+  *reinterpret_cast<uint2*>(p.out + off) = make_uint2(w0, w1);
+  if (!p.flow) return;
+  FlowStep step;
+  step.sigma = p.sigma;
+  step.renoise = p.sigma_next >= 0.0;
+  step.sigma_next = step.renoise ? p.sigma_next : 0.0;
+  step.one_minus_next = __dsub_rn(1.0, step.sigma_next);
+  const bool cfg = p.v_cond != nullptr;
+  const uint2 xv = __ldg(reinterpret_cast<const uint2*>(p.xt + off));
+  const uint2 ev = step.renoise ? __ldg(reinterpret_cast<const uint2*>(p.eps + off)) : make_uint2(0, 0);
+  const uint2 cv = cfg ? __ldg(reinterpret_cast<const uint2*>(p.v_cond + off)) : make_uint2(0, 0);
+  const uint32_t xw[2] = {xv.x, xv.y}, ew[2] = {ev.x, ev.y}, cw[2] = {cv.x, cv.y}, vw[2] = {w0, w1};
+  uint32_t o0[2], o1[2];
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    uint16_t a0, a1, b0 = 0, b1 = 0;
+    if (cfg) {
+      step.apply_cfg_bits(xw[q], cw[q], vw[q], ew[q], p.cfg_scale, a0, b0);
+      step.apply_cfg_bits(xw[q] >> 16, cw[q] >> 16, vw[q] >> 16, ew[q] >> 16, p.cfg_scale, a1, b1);
+    } else {
+      step.apply_bits(xw[q], vw[q], ew[q], a0, b0);
+      step.apply_bits(xw[q] >> 16, vw[q] >> 16, ew[q] >> 16, a1, b1);
+    }
+    o0[q] = static_cast<uint32_t>(a0) | (static_cast<uint32_t>(a1) << 16);
+    o1[q] = static_cast<uint32_t>(b0) | (static_cast<uint32_t>(b1) << 16);
+  }
+  *reinterpret_cast<uint2*>(p.x0 + off) = make_uint2(o0[0], o0[1]);
+  if (step.renoise) *reinterpret_cast<uint2*>(p.xt_next + off) = make_uint2(o1[0], o1[1]);
+}
+
 }  // namespace
 
 // Key streams of at most this many 128-key tiles take the short-stream form.
 constexpr int kShortStreamTiles = 16;
+// A unit is split in two only if each half keeps at least this many key tiles.
+constexpr int kSplitMinTiles = 16;
 
 cudaError_t launch_attention(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_vc,
                              const CUtensorMap& tm_vn, const CUtensorMap& tm_o, const AttnParams& p,
@@ -925,14 +1011,32 @@ cudaError_t launch_attention(const CUtensorMap& tm_q, const CUtensorMap& tm_k, c
     }
   }
   const int n_qb = (p.Lq + 2 * kBM - 1) / (2 * kBM);
+  const long long units = static_cast<long long>(n_qb) * p.H;
+  const int sm = sms[dev] > 0 ? sms[dev] : 1;
   if (p.n_tiles <= kShortStreamTiles) {
-    const long long units = static_cast<long long>(n_qb) * p.H;
-    const unsigned grid = static_cast<unsigned>(std::min<long long>(units, sms[dev] > 0 ? sms[dev] : 1));
+    const unsigned grid = static_cast<unsigned>(std::min<long long>(units, sm));
     chunk_attention_short_kernel<<<grid, kThreads, kSmemBytesShort, stream>>>(tm_q, tm_k, tm_vc, tm_vn, tm_o, p);
-  } else {
-    dim3 grid(n_qb, p.H);
-    chunk_attention_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_q, tm_k, tm_vc, tm_vn, p);
+    return cudaGetLastError();
   }
+  // One CTA per unit, all of equal length: with U units on the SMs the last wave runs
+  // U mod SMs of them while the other SMs idle. When that tail is at most half a wave (and
+  // the stream long enough), its units run as two CTAs over half the keys each, so the tail
+  // takes half as long; a combine launch then merges the halves.
+  AttnParams q = p;
+  q.split_first = static_cast<int>(units);
+  q.split_tiles = 0;
+  const long long tail = units % sm;
+  if (p.part != nullptr && units > sm && tail > 0 && 2 * tail <= sm && 2 * tail <= p.part_ctas &&
+      p.n_tiles >= 2 * kSplitMinTiles) {
+    q.split_first = static_cast<int>(units - tail);
+    q.split_tiles = p.n_tiles / 2;
+  }
+  const unsigned grid = static_cast<unsigned>(q.split_first + 2 * (units - q.split_first));
+  chunk_attention_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_q, tm_k, tm_vc, tm_vn, q);
+  err = cudaGetLastError();
+  if (err != cudaSuccess || q.split_first == units) return err;
+  const long long warps = (units - q.split_first) * (2 * kBM);
+  attention_combine_kernel<<<static_cast<unsigned>((warps + 7) / 8), 256, 0, stream>>>(q);
   return cudaGetLastError();
 }
 

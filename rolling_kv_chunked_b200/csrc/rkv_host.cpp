@@ -71,6 +71,10 @@ struct rkv_ctx {
   float2* tab_h = nullptr;
   float2* tab_w = nullptr;
   unsigned* status = nullptr;
+  // fp32 partial rows of the key-split last wave of long-stream attention launches
+  // (one CTA per SM, 256 rows each; shared by the handle's layers, whose calls run in order)
+  float* part = nullptr;
+  int part_ctas = 0;
   unsigned long long wait_ns = 2000000000ull;
   std::vector<Layer> L;
   // optional per-launch timing of the attention kernel
@@ -295,6 +299,16 @@ RKV_API int rkv_create(int layers, int H, int d, int tokens_per_frame, int windo
   int rc = RKV_OK;
   if (cudaMalloc(&h->status, sizeof(unsigned)) != cudaSuccess || cudaMemset(h->status, 0, sizeof(unsigned)) != cudaSuccess)
     rc = RKV_ERR_CUDA;
+  if (rc == RKV_OK) {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0 ||
+        cudaMalloc(&h->part, static_cast<size_t>(sms) * 2 * rkv::kQueryBox * rkv::kPartRow * sizeof(float)) !=
+            cudaSuccess)
+      rc = RKV_ERR_CUDA;
+    else
+      h->part_ctas = sms;
+  }
   for (int l = 0; l < layers && rc == RKV_OK; ++l) {
     Layer& L = h->L[l];
     L.slot_frame.assign(window_frames, -1);
@@ -536,6 +550,8 @@ int chunk_attention_impl(rkv_handle h, int layer, const void* q, const void* k, 
   }
   ap.status = h->status;
   ap.wait_limit_ns = h->wait_ns;
+  ap.part = h->part;
+  ap.part_ctas = h->part_ctas;
   CUtensorMap tm_vn, tm_o;
   if (!encode_token_major(&tm_vn, v, C * T, h->H, rkv::kKeyBox) ||
       !encode_token_major(&tm_o, out, C * T, h->H, rkv::kQueryBox))
@@ -657,6 +673,8 @@ RKV_API int rkv_cross_attention(rkv_handle h, int layer, const void* q, void* ou
   ap.sigma_next = -1.0;
   ap.status = h->status;
   ap.wait_limit_ns = h->wait_ns;
+  ap.part = h->part;
+  ap.part_ctas = h->part_ctas;
   CUtensorMap tm_q, tm_o;
   if (!encode_token_major(&tm_q, q, n_tokens, h->H, rkv::kQueryBox) ||
       !encode_token_major(&tm_o, out, n_tokens, h->H, rkv::kQueryBox))
@@ -878,6 +896,7 @@ RKV_API int rkv_destroy(rkv_handle h) {
   cudaFree(h->tab_h);
   cudaFree(h->tab_w);
   cudaFree(h->status);
+  cudaFree(h->part);
   delete h;
   return RKV_OK;
 }

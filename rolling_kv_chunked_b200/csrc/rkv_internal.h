@@ -98,7 +98,18 @@ struct AttnParams {
   double cfg_scale;
   unsigned* status;
   unsigned long long wait_limit_ns;
+  // Scratch for splitting the last, partial wave of a long key stream into two key halves
+  // (launch_attention decides; null: never split): fp32 partial rows of kPartRow floats
+  // (O unnormalised, then the reference and the sum), room for part_ctas CTAs of 256 rows.
+  float* part;
+  int part_ctas;
+  // set by launch_attention: units u >= split_first (u = head * query blocks + block) run as
+  // two CTAs over key tiles [0, split_tiles) and [split_tiles, n_tiles)
+  int split_first;
+  int split_tiles;
 };
+
+constexpr int kPartRow = 132;  // floats per partial row: 128 of O, the reference, the sum, 2 unused
 
 cudaError_t launch_attention(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_vc,
                              const CUtensorMap& tm_vn, const CUtensorMap& tm_o, const AttnParams& p,

@@ -634,3 +634,40 @@ def test_fused_flow_with_more_units_than_sms():
         ref = orc.chunk_attention(qb, kb, vb, cfg.C, chunk, True, rows=rows, heads=heads)
         assert_close(to_bits(out)[rows][:, heads], ref, f"chunk {chunk}")
     h.close()
+
+
+def test_split_last_wave_with_fused_flow():
+    """16 heads x 10 query blocks = 160 units of a 50-tile key stream: 148 run whole, the last
+    12 (heads 14 and 15) as two CTAs over half the keys each plus a combine launch. The fused
+    x0 / renoise step must equal the oracle's step on the stored output bit for bit (also on
+    the split units), and the output of a split head and of a whole one must match the oracle
+    on sampled rows."""
+    cfg = Config("split", 18, H=16, grid_h=32, grid_w=40, C=2, W=5, S=1, rope_mode=ABS, chunks=1)
+    h = rkv.RollingKV(1, cfg.H, 128, cfg.T, cfg.W, cfg.S, cfg.rope_mode)
+    h.set_rope_grid(cfg.grid_h, cfg.grid_w)
+    orc = OracleLayer(cfg.H, 128, cfg.T, cfg.grid_h, cfg.grid_w, cfg.W, cfg.S, cfg.rope_mode)
+    kw, vw = (dev_tensor(torch, cfg, 0, -1, 0, t, 3 * cfg.T) for t in ("k", "v"))
+    h.write_chunk(0, kw, vw, 3, 0)
+    orc.write_chunk(to_bits(kw), to_bits(vw), 3, 0)
+    Lq, n = cfg.Lq, cfg.Lq * cfg.H * 128
+    q, k, v = (dev_tensor(torch, cfg, 0, 0, 0, t, Lq) for t in ("q", "k", "v"))
+    xt = _dev_bits(synth.stream_key(0, 18, 1), n)
+    eps = _dev_bits(synth.stream_key(0, 18, 2), n)
+    for s, sn in [(1.0, 0.75), (0.25, -1.0)]:
+        out = torch.empty((Lq, cfg.H, 128), dtype=torch.bfloat16, device="cuda")
+        x0 = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+        xn = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+        h.chunk_attention(0, q, k, v, out, cfg.C, 3, False,
+                          flow=dict(xt=xt, eps=eps, sigma=s, sigma_next=sn, x0_out=x0,
+                                    xt_next_out=xn if sn >= 0 else None))
+        torch.cuda.synchronize()
+        assert h.poll_device_status() == rkv.OK
+        rx0, rxn = oflow.x0_renoise_bf16(to_bits(xt), to_bits(out).reshape(-1), to_bits(eps), s, sn)
+        assert np.array_equal(to_bits(x0), rx0)
+        if sn >= 0:
+            assert np.array_equal(to_bits(xn), rxn)
+    rows = sample_rows(Lq, n=64, seed=18)
+    heads = [0, 15]
+    ref = orc.chunk_attention(to_bits(q), to_bits(k), to_bits(v), cfg.C, 3, False, rows=rows, heads=heads)
+    assert_close(to_bits(out)[rows][:, heads], ref, "split last wave")
+    h.close()
