@@ -211,6 +211,20 @@ def visible_keys(cfg, committed, f0):
     return sum(n for _, _, n, _ in rkv.plan_window(cfg["W"], cfg["S"], committed, cfg["C"], f0)) * T
 
 
+def attention_launches(cfg, committed, f0, sms):
+    """Kernel launches of one attention call's attention part: 1, or 2 when the library runs the
+    long-stream launch's partial last wave split by keys (then a combine launch follows). The
+    same rule as the library's launcher: more units than SMs, a tail of at most half the SMs,
+    and at least 32 key tiles."""
+    import rolling_kv_chunked_b200 as rkv
+    T = cfg["gh"] * cfg["gw"]
+    Lq = cfg["C"] * T
+    tiles = sum(-(-n * T // 128) for _, _, n, _ in rkv.plan_window(cfg["W"], cfg["S"], committed, cfg["C"], f0))
+    units = -(-Lq // 256) * cfg["H"]
+    tail = units % sms
+    return 2 if tiles > 16 and tiles >= 32 and units > sms and 0 < tail and 2 * tail <= sms else 1
+
+
 # a timed region at least this long is compared with the sustained (power-capped) bf16 peak;
 # a shorter one with the burst peak
 SUSTAINED_REGION_S = 1.0
@@ -344,11 +358,16 @@ def measure_workload(args, name, headline):
     if h.poll_device_status(sp) != rkv.OK:
         raise RuntimeError("device wait expired during warm-up")
 
-    # FLOPs of the attention launches in the timed region (unmasked visible keys)
+    # FLOPs of the attention launches in the timed region (unmasked visible keys), and our
+    # kernel launches there: per call the RoPE pre-pass and the attention (plus a combine
+    # launch when its last wave is split), and the commit's write-back once per step
     flops = 0.0
+    launches = 0
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
     f = state["f0"]
     for _ in range(args.steps):
         flops += n_layers * 5 * 4.0 * H * 128 * Lq * visible_keys(cfg, f, f)
+        launches += n_layers * (5 * (1 + attention_launches(cfg, f, f, sms)) + 1)
         f += C
 
     if world > 1:
@@ -447,7 +466,7 @@ def measure_workload(args, name, headline):
         "e2e": e2e,
         "hbm_kernels": hbm,
         "cross_attention": cross,
-        "gpu_launches": 11 * n_layers * args.steps,
+        "gpu_launches": launches,
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -592,7 +611,9 @@ def run_cfg(args):
         "hbm_kernels": {"flow_cfg_x0_renoise": {"bytes_per_launch": 12 * n, "GB/s": ep_gbs,
                                                 "frac_of_hbm": ep_gbs / pk["hbm_gbs"]},
                         "peak_hbm_gbs": pk["hbm_gbs"], "peak_source": pk_kind},
-        "gpu_launches": (2 * CFG_STEPS * 2 + 2 * 2) * args.steps,
+        "gpu_launches": (2 * CFG_STEPS * (1 + attention_launches(
+            cfg, W, W, torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count))
+            + 2 * 2) * args.steps,
         "clocks": clk,
     }
     for h in hs:
